@@ -1,0 +1,282 @@
+"""CPU oracle for block-scaled FP4 quantization and the block-scaled FP4 GEMM.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package; the library package
+(``fp4_block_scaled_h16_b200``) never does, and this package never imports it.
+
+The quantizer is plain C (``fp4_oracle.c``, compiled with FMA contraction off),
+called through ctypes; the GEMM is the plain definition: dequantize both
+operands exactly into float64 and take their float64 matrix product, with the
+per-element bound sum_k |a_ik * b_jk| beside it.
+
+Sources (page titles, sections):
+  * E2M1 grid, RTNE, shrinkage: "Ripensare il Bias di Shrinkage nel Pretraining
+    di LLM in FP4", Problematica, Metodologia 1; UFP4: Metodologia 2.
+  * MXFP4, H16/H32, random Hadamard: "Pre-addestramento di Modelli Linguistici
+    di Grandi Dimensioni con MXFP4", Metodologia.
+  * NVFP4 16-groups, double block 128/16, SR, 1x16 transposed groups:
+    "TetraJet-v2", section 2.A.
+  * Fprop / Dgrad / Wgrad GEMMs on FP4 operands: the MXFP4 page, Metodologia.
+
+Parity unpinned (readings the pages do not fix, pinned only between this
+oracle and the CUDA path): the binary32 operation order of the NVFP4 / UFP4 /
+double-block scale, the H32 normalisation constant, the Philox counter layout
+for SR and the random signs.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+MXFP4, NVFP4, UFP4 = 0, 1, 2
+RTNE, SR = 0, 1
+ROT_NONE, ROT_H16, ROT_H32, ROT_RH16, ROT_RH32 = 0, 1, 2, 3, 4
+IN_F32, IN_BF16 = 0, 1
+
+E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def build(force: bool = False) -> str:
+    """Compile fp4_oracle.c into liboracle.so next to it (gcc, no FMA contraction)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math",
+                           "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i64, u64, u32, f32, i32 = (ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint32,
+                                   ctypes.c_float, ctypes.c_int)
+        L.orc_philox4x32_10.argtypes = [P, P, P]
+        L.orc_rht_signs.argtypes = [u64, i32, P]
+        L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_value.restype = ctypes.c_double
+        L.orc_ufp4_value.argtypes = [ctypes.c_uint8]
+        L.orc_ufp4_value.restype = ctypes.c_double
+        L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_value.restype = ctypes.c_double
+        L.orc_e4m3_encode.argtypes = [f32]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e2m1_rtne_index.argtypes = [f32]
+        L.orc_ufp4_rtne_index.argtypes = [f32]
+        L.orc_rotate_block.argtypes = [P, i32, P]
+        L.orc_c32.restype = f32
+        L.orc_tensor_amax.argtypes = [P, i32, i64, i64, i64, i32, i32, u64, i64, i64]
+        L.orc_tensor_amax.restype = f32
+        L.orc_tensor_scale.argtypes = [f32, i32]
+        L.orc_tensor_scale.restype = f32
+        L.orc_quantize_lines.argtypes = [P, i32, i64, i64, i64, i32, i32, i32, i32, i32,
+                                         u64, u32, f32, i64, i64, P, P, P]
+        L.orc_dequantize.argtypes = [P, P, P, f32, i64, i64, i32, i32, P]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_threads() -> int:
+    return max(1, min(os.cpu_count() or 1, 32))
+
+
+# --------------------------------------------------------------------------- scalars
+
+def philox4x32_10(ctr, key) -> np.ndarray:
+    c = np.asarray(ctr, dtype=np.uint32)
+    k = np.asarray(key, dtype=np.uint32)
+    out = np.zeros(4, dtype=np.uint32)
+    lib().orc_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def rht_signs(seed: int, n: int) -> np.ndarray:
+    d = np.zeros(n, dtype=np.float32)
+    lib().orc_rht_signs(seed, n, _ptr(d))
+    return d
+
+
+def rotate_block(x, signs=None) -> np.ndarray:
+    b = np.array(x, dtype=np.float32)
+    d = None if signs is None else np.ascontiguousarray(signs, dtype=np.float32)
+    lib().orc_rotate_block(_ptr(b), len(b), None if d is None else _ptr(d))
+    return b
+
+
+def c32() -> float:
+    return lib().orc_c32()
+
+
+def e4m3_value(code: int) -> float:
+    return lib().orc_e4m3_value(code)
+
+
+def e4m3_encode(s: float) -> int:
+    return lib().orc_e4m3_encode(s)
+
+
+def e2m1_value(code: int) -> float:
+    return lib().orc_e2m1_value(code)
+
+
+def ufp4_value(code: int) -> float:
+    return lib().orc_ufp4_value(code)
+
+
+def e2m1_rtne_index(u: float) -> int:
+    return lib().orc_e2m1_rtne_index(u)
+
+
+def ufp4_rtne_index(u: float) -> int:
+    return lib().orc_ufp4_rtne_index(u)
+
+
+def tensor_scale(amax: float, fmt: int) -> float:
+    return lib().orc_tensor_scale(amax, fmt)
+
+
+# --------------------------------------------------------------------------- tensors
+
+def _as_input(x: np.ndarray):
+    if x.dtype == np.float32:
+        return IN_F32
+    if x.dtype == np.uint16:           # bfloat16 bit patterns
+        return IN_BF16
+    raise TypeError("oracle input must be float32 or uint16 (bf16 bits), got %s" % x.dtype)
+
+
+def _chunks(l0: int, l1: int, threads: int):
+    n = l1 - l0
+    if n <= 0:
+        return []
+    step = max(1, -(-n // (threads * 4)))
+    return [(a, min(a + step, l1)) for a in range(l0, l1, step)]
+
+
+def tensor_amax(x: np.ndarray, axis: int, rotation: int = ROT_NONE, seed: int = 0,
+                C: int | None = None, threads: int | None = None) -> float:
+    """max |y| over the rotated tensor (rotation along the quantization axis)."""
+    x = np.ascontiguousarray(x)
+    dt = _as_input(x)
+    R, ld = x.shape
+    C = ld if C is None else C
+    lines = R if axis == 1 else C
+    threads = threads or default_threads()
+    L = lib()
+
+    def run(rng):
+        return L.orc_tensor_amax(_ptr(x), dt, R, C, ld, axis, rotation, seed, rng[0], rng[1])
+
+    parts = _chunks(0, lines, threads)
+    if not parts:
+        return 0.0
+    with ThreadPoolExecutor(threads) as ex:
+        return float(max(ex.map(run, parts)))
+
+
+def quantize(x: np.ndarray, fmt: int, rounding: int = RTNE, rotation: int = ROT_NONE,
+             axis: int = 1, double_block: bool = False, seed: int = 0, tensor_id: int = 0,
+             amax: float | None = None, lines=None, C: int | None = None,
+             threads: int | None = None) -> dict:
+    """Quantize a row-major [R, ld] tensor (logical [R, C]) along ``axis``.
+
+    Returns a dict with ``codes`` [L, K/2] uint8, ``scales`` [L, K/blk] uint8
+    (row-major), ``outer`` [L, K/128] float32 (double block), ``tensor_scale``
+    (NV/UFP4 without double block), ``amax`` and ``lines`` (the line indices).
+    ``lines`` selects a subset of output lines (sampling); the tensor amax is
+    always taken over the whole tensor unless ``amax`` is given.
+    """
+    x = np.ascontiguousarray(x)
+    dt = _as_input(x)
+    R, ld = x.shape
+    C = ld if C is None else C
+    K = C if axis == 1 else R
+    nlines = R if axis == 1 else C
+    blk = 32 if fmt == MXFP4 else 16
+    threads = threads or default_threads()
+    needs_ts = fmt in (NVFP4, UFP4) and not double_block
+    if needs_ts and amax is None:
+        amax = tensor_amax(x, axis, rotation, seed, C=C, threads=threads)
+    ts = tensor_scale(amax, fmt) if needs_ts else 1.0
+    if lines is None:
+        idx = np.arange(nlines, dtype=np.int64)
+    else:
+        idx = np.asarray(lines, dtype=np.int64)
+    n = len(idx)
+    codes = np.zeros((n, K // 2), dtype=np.uint8)
+    scales = np.zeros((n, K // blk), dtype=np.uint8)
+    outer = np.zeros((n, max(K // 128, 0)), dtype=np.float32)
+    # runs of consecutive line indices, each processed by one C call
+    runs = []
+    s = 0
+    for t in range(1, n + 1):
+        if t == n or idx[t] != idx[t - 1] + 1:
+            runs.append((s, t))
+            s = t
+    work = []
+    for (a, b) in runs:
+        for (u, v) in _chunks(a, b, threads):
+            work.append((u, v))
+    L = lib()
+
+    def run(uv):
+        u, v = uv
+        rc = L.orc_quantize_lines(_ptr(x), dt, R, C, ld, fmt, rounding, rotation, axis,
+                                  int(double_block), seed, tensor_id, ts,
+                                  int(idx[u]), int(idx[u]) + (v - u),
+                                  _ptr(codes[u:v]), _ptr(scales[u:v]), _ptr(outer[u:v]))
+        if rc:
+            raise ValueError("oracle rejected the shape/format combination (code %d)" % rc)
+
+    if work:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(run, work))
+    return dict(codes=codes, scales=scales, outer=outer if double_block else None,
+                tensor_scale=ts if needs_ts else None, amax=amax, lines=idx, K=K,
+                format=fmt, double_block=bool(double_block))
+
+
+def dequantize(q: dict) -> np.ndarray:
+    """Exact float64 values of a quantized tensor: q * s_b * (s_t or s_o)."""
+    codes = np.ascontiguousarray(q["codes"])
+    scales = np.ascontiguousarray(q["scales"])
+    n, K = codes.shape[0], q["K"]
+    outer = q.get("outer")
+    outer = np.ascontiguousarray(outer if outer is not None else np.zeros((n, 1), np.float32))
+    ts = q.get("tensor_scale") or 1.0
+    out = np.zeros((n, K), dtype=np.float64)
+    rc = lib().orc_dequantize(_ptr(codes), _ptr(scales), _ptr(outer), ts, n, K, q["format"],
+                              int(q["double_block"]), _ptr(out))
+    if rc:
+        raise ValueError("oracle dequantize rejected the shape (code %d)" % rc)
+    return out
+
+
+def gemm(qa: dict, qb: dict):
+    """C64 = deq(A) @ deq(B)^T in float64 and the bound sum_k |a_ik b_jk|.
+
+    A is [M, K] and B is [N, K], both K-major quantized tensors (their
+    lines run along K), as the Fprop / Dgrad / Wgrad GEMMs consume them.
+    """
+    a = dequantize(qa)
+    b = dequantize(qb)
+    return a @ b.T, np.abs(a) @ np.abs(b).T
