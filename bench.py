@@ -1,0 +1,358 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled FP4 hot path on B200.
+
+One step = one pass of the whole path over one batch: the NVFP4 Fprop of the
+Llama-3.1-8B QKV projection at 8192 tokens -- rotated-tensor amax and fused
+H16-rotate/scale/round/pack quantization of X [8192, 4096] and of
+W [6144, 4096] (bf16), then the block-scaled FP4 GEMM Y = X W^T
+(8192 x 6144 x 4096, bf16 out).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp4|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU under torchrun,
+each rank runs its own independent problem (weak scaling, no collective on the
+data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp4_block_scaled_h16_b200 import workloads  # noqa: E402
+
+METRIC = "FP4 quantize GB/s and block-scaled FP4 GEMM TFLOPS (% of B200 roofline)"
+M, N, K = workloads.TOKENS, workloads.QKV_OUT, workloads.HIDDEN
+WORKLOAD = "nvfp4_fprop_qkv_%dx%dx%d" % (M, N, K)
+GEMM_FLOP = 2.0 * M * N * K
+L2_FLUSH_BYTES = 256 << 20
+# algorithmic bytes per element (bf16 in): amax pass reads 2 B; the quantize
+# pass reads 2 B and writes 0.5 B of codes + 1/16 B of E4M3 scale
+AMAX_BPE = 2.0
+QUANT_BPE = 2.0 + 0.5 + 1.0 / 16.0
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained"),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": names}
+
+
+# ------------------------------------------------------------------------ GPU arm
+
+class Fprop:
+    """Device buffers and the step of the NVFP4 Fprop workload."""
+
+    def __init__(self, fp4, X, W, device):
+        self.fp4 = fp4
+        self.X, self.W = X.to(device), W.to(device)
+        self.qx = fp4.alloc_qtensor(M, K, fp4.FP4_NVFP4, device=device)
+        self.qw = fp4.alloc_qtensor(N, K, fp4.FP4_NVFP4, device=device)
+        self.ax = torch.empty(1, dtype=torch.float32, device=device)
+        self.aw = torch.empty(1, dtype=torch.float32, device=device)
+        self.C = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.launches_per_step = 5     # amax X, quantize X, amax W, quantize W, GEMM
+
+    def quant(self, x, q, amax):
+        f = self.fp4
+        f.fp4_amax(x, f.FP4_IN_BF16, x.shape[0], x.shape[1], x.shape[1], f.FP4_ROT_H16, 1, 0, amax)
+        f.quantize(x, f.FP4_NVFP4, f.FP4_RTNE, f.FP4_ROT_H16, axis=1, tensor_amax=amax, out=q)
+
+    def gemm(self):
+        self.fp4.gemm(self.qx, self.qw, self.fp4.FP4_OUT_BF16, out=self.C)
+
+    def step(self, ev=None):
+        if ev:
+            ev[0].record()
+        self.quant(self.X, self.qx, self.ax)
+        if ev:
+            ev[1].record()
+        self.quant(self.W, self.qw, self.aw)
+        if ev:
+            ev[2].record()
+        self.gemm()
+        if ev:
+            ev[3].record()
+
+
+def run_gpu(args, rank, world, device):
+    from fp4_block_scaled_h16_b200 import fp4
+    peaks = measured_peaks()
+    d = workloads.nvfp4_fprop_qkv(seed=rank)
+    w = Fprop(fp4, d["X"], d["W"], device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        w.step()
+    torch.cuda.synchronize()
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clocks:
+        for i in range(args.steps):
+            flush.zero_()                       # L2 flush, outside the timed events
+            w.step(evs[i])
+        torch.cuda.synchronize()
+    barrier()
+    qx = [e[0].elapsed_time(e[1]) for e in evs]
+    qw = [e[1].elapsed_time(e[2]) for e in evs]
+    gm = [e[2].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    total_ms = sum(step_ms)
+    status = fp4.fp4_last_error()
+
+    # per-kernel split of the quantize calls (amax pass vs quantize pass), timed
+    # separately on a second pass so the main loop stays one stream of launches
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    amax_ms, quant_ms = [], []
+    for _ in range(max(3, min(args.steps, 20))):
+        flush.zero_()
+        ev_a[0].record()
+        fp4.fp4_amax(w.X, fp4.FP4_IN_BF16, M, K, K, fp4.FP4_ROT_H16, 1, 0, w.ax)
+        ev_a[1].record()
+        fp4.quantize(w.X, fp4.FP4_NVFP4, fp4.FP4_RTNE, fp4.FP4_ROT_H16, axis=1, tensor_amax=w.ax, out=w.qx)
+        ev_a[2].record()
+        torch.cuda.synchronize()
+        amax_ms.append(ev_a[0].elapsed_time(ev_a[1]))
+        quant_ms.append(ev_a[1].elapsed_time(ev_a[2]))
+
+    # end to end through the public API: pinned host inputs in, result out
+    e2e_steps = max(3, min(args.steps, 20))
+    hX = d["X"].pin_memory()
+    hW = d["W"].pin_memory()
+    hC = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for _ in range(e2e_steps):
+        flush.zero_()
+        e0.record()
+        w.X.copy_(hX, non_blocking=True)
+        w.W.copy_(hW, non_blocking=True)
+        w.step()
+        hC.copy_(w.C, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+
+    t = torch.tensor([total_ms, statistics.mean(e2e_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_max, e2e_max = float(t[0]), float(t[1])
+    if rank != 0:
+        return None
+
+    ms_per_step = total_max / args.steps
+    value = world * args.steps * GEMM_FLOP / (total_max * 1e-3) / 1e12
+    gemm_ms = statistics.mean(gm)
+    fp4_peak = peaks["bf16"] * 4.0      # nominal dense fp4 / bf16 ratio (9 / 2.25 PFLOP/s)
+    achieved = GEMM_FLOP / (gemm_ms * 1e-3) / 1e12
+    bpe_x = M * K
+    comp = {
+        "amax_X": {"ms": statistics.mean(amax_ms), "gbs": AMAX_BPE * bpe_x / (statistics.mean(amax_ms) * 1e6)},
+        "quantize_X": {"ms": statistics.mean(quant_ms), "gbs": QUANT_BPE * bpe_x / (statistics.mean(quant_ms) * 1e6)},
+        "amax+quantize_X": {"ms": statistics.mean(qx), "gbs_2read": (AMAX_BPE + QUANT_BPE) * M * K / (statistics.mean(qx) * 1e6)},
+        "amax+quantize_W": {"ms": statistics.mean(qw), "gbs_2read": (AMAX_BPE + QUANT_BPE) * N * K / (statistics.mean(qw) * 1e6)},
+        "gemm": {"ms": gemm_ms, "tflops": achieved},
+    }
+    for k in ("amax_X", "quantize_X"):
+        comp[k]["frac_hbm"] = comp[k]["gbs"] / peaks["hbm"]
+    for k in ("amax+quantize_X", "amax+quantize_W"):
+        comp[k]["frac_hbm"] = comp[k]["gbs_2read"] / peaks["hbm"]
+    comp["gemm"]["frac_fp4"] = achieved / fp4_peak
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 scales) -> f32 accumulate; quantizer f32",
+        "data": "synthetic (seeded: X N(0,1) with 8 outlier channels x64, W N(0,0.02); bf16)",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "format": "NVFP4",
+                   "rotation": "H16", "rounding": "RTNE", "out": "bf16",
+                   "value_is": "GEMM FLOP of the step / whole step time (amax + quantize X, W + GEMM)",
+                   "l2": "flushed between steps (256 MiB write outside the timed events)",
+                   "parallelism": "independent problem per GPU" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_kernel (NVFP4, 128x256 tile)",
+                     "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / fp4_peak, 4), "traffic": None,
+                     "peak_is": "%s bf16 burst %.1f TFLOP/s x 4 (nominal fp4/bf16)" % (peaks["src"], peaks["bf16"])},
+        "components": comp,
+        "e2e": {"value": round(world * GEMM_FLOP / (e2e_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(d["X"].numel() * 2 + d["W"].numel() * 2),
+                "d2h_bytes_per_step": int(M * N * 2), "ms_per_step": round(e2e_max, 4)},
+        "gpu_launches": w.launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "device_status": fp4.fp4_status_string(status),
+    }
+    return line
+
+
+# ------------------------------------------------------------------------ oracle arm
+
+def oracle_slab_time(d, rows):
+    """Oracle time of the step restricted to `rows` rows of X and of W,
+    extrapolated to the whole workload (seconds), and the threads it used."""
+    import oracle
+    X = workloads.bf16_bits(d["X"][:rows])
+    W = workloads.bf16_bits(d["W"][:rows])
+    t0 = time.perf_counter()
+    ax = oracle.tensor_amax(X, 1, oracle.ROT_H16)
+    t1 = time.perf_counter()
+    qx = oracle.quantize(X, oracle.NVFP4, rotation=oracle.ROT_H16, amax=ax)
+    t2 = time.perf_counter()
+    aw = oracle.tensor_amax(W, 1, oracle.ROT_H16)
+    t3 = time.perf_counter()
+    qw = oracle.quantize(W, oracle.NVFP4, rotation=oracle.ROT_H16, amax=aw)
+    t4 = time.perf_counter()
+    oracle.gemm(qx, qw)
+    t5 = time.perf_counter()
+    full = ((t2 - t0) * M / rows + (t4 - t2) * N / rows + (t5 - t4) * (M * N) / (rows * rows))
+    return full, oracle.default_threads()
+
+
+def cpu_baseline(d, target_s=10.0):
+    rows = 64
+    t, cores = oracle_slab_time(d, rows)
+    # grow the slab towards ~target_s of CPU work
+    spent = t * rows / M
+    if spent < target_s / 4:
+        rows = int(min(1024, rows * target_s / 2 / max(spent, 1e-3)))
+        rows = max(64, rows - rows % 16)
+        t, cores = oracle_slab_time(d, rows)
+    value = GEMM_FLOP / t / 1e12
+    return {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": "%d rows of X and of W: amax + quantize (NVFP4, H16) and the float64 GEMM of "
+                      "the %dx%d slab, each part extrapolated to the full 8192x6144x4096 step" % (rows, rows, rows)}
+
+
+def run_reference(args):
+    """The oracle, as it stands, timed on the host cores on a bounded sample."""
+    d = workloads.nvfp4_fprop_qkv(seed=0)
+    budget_s = 120.0
+    rows = 64
+    t_cal, cores = oracle_slab_time(d, rows)
+    per_step_real = t_cal * rows / M + t_cal * rows * rows / (M * N)   # rough real seconds per slab step
+    steps = args.steps + args.warmup
+    if per_step_real * steps > budget_s:
+        rows = 16
+    times = []
+    for i in range(args.warmup + args.steps):
+        t, cores = oracle_slab_time(d, rows)
+        if i >= args.warmup:
+            times.append(t)
+    ms = statistics.mean(times) * 1e3
+    value = GEMM_FLOP / (ms * 1e-3) / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizer, f64 GEMM (CPU oracle)",
+        "data": "synthetic (same seeded workload)",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "format": "NVFP4", "rotation": "H16",
+                   "rounding": "RTNE", "out": "f64"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "per step: %d rows of X and W through the whole step, extrapolated" % rows},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["fp4", "reference"], default="fp4")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    line = run_gpu(args, rank, world, device)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(workloads.nvfp4_fprop_qkv(seed=0))
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,297 @@
+// fp4_api.cu -- the extern "C" entry points of libfp4.so (declared in
+// include/fp4.h): argument validation, the host-side Philox key schedule and
+// sign mask, and the launches.  The library allocates no device memory.
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fp4.h"
+#include "internal.h"
+
+namespace fp4 {
+
+__device__ unsigned int g_error_word;    // FP4_ERR_TIMEOUT etc., set by kernels
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices];
+int g_arch_ok[kMaxDevices];               // 0 unknown, 1 sm_100, -1 other
+unsigned int* g_err_ptr[kMaxDevices];
+std::mutex g_mu;
+uint32_t g_wait_limit = 1u << 20;
+
+// Philox4x32-10 on the host, for the random-sign word and the round keys
+// (Salmon et al., SC'11: multipliers 0xD2511F53 / 0xCD9E8D57, Weyl key bumps
+// 0x9E3779B9 / 0xBB67AE85).
+PhiloxKeys make_keys(uint64_t seed) {
+    PhiloxKeys k;
+    uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
+    for (int r = 0; r < 10; ++r) {
+        k.k0[r] = a;
+        k.k1[r] = b;
+        a += 0x9E3779B9u;
+        b += 0xBB67AE85u;
+    }
+    return k;
+}
+
+uint32_t philox_word0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, const PhiloxKeys& k) {
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0, p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k.k0[r];
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k.k1[r];
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
+        c0 = n0;
+        c2 = n2;
+    }
+    return c0;
+}
+
+int rot_size(int rotation) {
+    return (rotation == FP4_ROT_H16 || rotation == FP4_ROT_RH16) ? 16
+         : (rotation == FP4_ROT_H32 || rotation == FP4_ROT_RH32) ? 32 : 0;
+}
+
+uint32_t sign_mask_of(int rotation, uint64_t seed) {
+    if (rotation != FP4_ROT_RH16 && rotation != FP4_ROT_RH32) return 0u;
+    const uint32_t w = philox_word0(0u, 0u, 0u, 1u, make_keys(seed));
+    return rotation == FP4_ROT_RH16 ? (w & 0xFFFFu) : w;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// current device is a usable sm_100 GPU; caches the SM count and error word
+fp4_status_t device_ready(int* dev_out) {
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess || n == 0) {
+        cudaGetLastError();
+        return FP4_ERR_NO_DEVICE;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP4_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_arch_ok[dev] == 0) {
+        int major = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FP4_ERR_CUDA;
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return FP4_ERR_CUDA;
+        g_err_ptr[dev] = static_cast<unsigned int*>(p);
+        g_sms[dev] = sms;
+        g_arch_ok[dev] = (major == 10) ? 1 : -1;
+    }
+    if (g_arch_ok[dev] != 1) return FP4_ERR_NO_DEVICE;
+    *dev_out = dev;
+    return FP4_OK;
+}
+
+}  // namespace
+
+int num_sms() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return (dev >= 0 && dev < kMaxDevices && g_sms[dev] > 0) ? g_sms[dev] : 148;
+}
+
+unsigned int* device_error_word() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return (dev >= 0 && dev < kMaxDevices) ? g_err_ptr[dev] : nullptr;
+}
+
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" {
+
+const char* fp4_status_string(fp4_status_t s) {
+    switch (s) {
+    case FP4_OK: return "FP4_OK";
+    case FP4_ERR_INVALID_ARG: return "FP4_ERR_INVALID_ARG";
+    case FP4_ERR_UNSUPPORTED_SHAPE: return "FP4_ERR_UNSUPPORTED_SHAPE";
+    case FP4_ERR_MISALIGNED: return "FP4_ERR_MISALIGNED";
+    case FP4_ERR_WORKSPACE: return "FP4_ERR_WORKSPACE";
+    case FP4_ERR_NO_DEVICE: return "FP4_ERR_NO_DEVICE";
+    case FP4_ERR_CUDA: return "FP4_ERR_CUDA";
+    case FP4_ERR_TIMEOUT: return "FP4_ERR_TIMEOUT";
+    case FP4_ERR_UNSUPPORTED: return "FP4_ERR_UNSUPPORTED";
+    }
+    return "FP4_ERR_UNKNOWN";
+}
+
+void fp4_set_wait_limit(uint32_t polls) { g_wait_limit = polls ? polls : (1u << 20); }
+
+size_t fp4_scales_bytes(int64_t lines, int64_t K, fp4_format_t format) {
+    if (lines <= 0 || K <= 0) return 0;
+    const int64_t blk = (format == FP4_MXFP4) ? 32 : 16;
+    const int64_t nb = K / blk;
+    return (size_t)(((lines + 127) / 128) * 128) * (size_t)(((nb + 3) / 4) * 4);
+}
+
+fp4_status_t fp4_quantize_workspace_size(fp4_format_t format, int double_block, int amax_given,
+                                         size_t* bytes) {
+    if (!bytes || format < FP4_MXFP4 || format > FP4_UFP4) return FP4_ERR_INVALID_ARG;
+    *bytes = (format != FP4_MXFP4 && !double_block && !amax_given) ? 256 : 0;
+    return FP4_OK;
+}
+
+static fp4_status_t check_input(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols,
+                                int64_t ld, fp4_rotation_t rotation, int axis) {
+    if (in_dtype != FP4_IN_F32 && in_dtype != FP4_IN_BF16) return FP4_ERR_INVALID_ARG;
+    if (rotation < FP4_ROT_NONE || rotation > FP4_ROT_RH32) return FP4_ERR_INVALID_ARG;
+    if (axis != 0 && axis != 1) return FP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return FP4_ERR_INVALID_ARG;
+    if (rows > 0 && cols > 0) {
+        if (!x) return FP4_ERR_INVALID_ARG;
+        const int64_t es = in_dtype == FP4_IN_BF16 ? 2 : 4;
+        if (!aligned16(x) || (ld * es) % 16) return FP4_ERR_MISALIGNED;
+    }
+    const int64_t K = axis ? cols : rows;
+    const int n = rot_size(rotation);
+    if (n && K % n) return FP4_ERR_UNSUPPORTED_SHAPE;
+    return FP4_OK;
+}
+
+fp4_status_t fp4_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                      fp4_rotation_t rotation, int axis, uint64_t seed, float* amax_out, void* stream) {
+    fp4_status_t st = check_input(x, in_dtype, rows, cols, ld, rotation, axis);
+    if (st != FP4_OK) return st;
+    if (!amax_out) return FP4_ERR_INVALID_ARG;
+    if ((uintptr_t)amax_out & 3u) return FP4_ERR_MISALIGNED;
+    int dev;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
+    if (rows == 0 || cols == 0) return FP4_OK;
+    QuantArgs a{};
+    a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
+    a.L = axis ? rows : cols;
+    a.K = axis ? cols : rows;
+    a.amax_out = reinterpret_cast<unsigned int*>(amax_out);
+    a.sign_mask = sign_mask_of(rotation, seed);
+    if (launch_amax(a, in_dtype == FP4_IN_BF16, rot_size(rotation), axis, s) != cudaSuccess) return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
+fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                          fp4_format_t format, fp4_rounding_t rounding, fp4_rotation_t rotation, int axis,
+                          int double_block, uint64_t seed, uint32_t tensor_id, const float* tensor_amax,
+                          uint8_t* codes, uint8_t* scales, float* outer_scales, float* tensor_scale,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    fp4_status_t st = check_input(x, in_dtype, rows, cols, ld, rotation, axis);
+    if (st != FP4_OK) return st;
+    if (format < FP4_MXFP4 || format > FP4_UFP4) return FP4_ERR_INVALID_ARG;
+    if (rounding != FP4_RTNE && rounding != FP4_SR) return FP4_ERR_INVALID_ARG;
+    if (double_block != 0 && double_block != 1) return FP4_ERR_INVALID_ARG;
+    if (double_block && format != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+    const int64_t K = axis ? cols : rows, L = axis ? rows : cols;
+    const int64_t blk = (format == FP4_MXFP4) ? 32 : 16;
+    if (K % blk) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (double_block && K % 128) return FP4_ERR_UNSUPPORTED_SHAPE;
+    const bool needs_ts = format != FP4_MXFP4 && !double_block;
+    const bool internal_amax = needs_ts && tensor_amax == nullptr;
+    const bool empty = (L == 0 || K == 0);
+    if (!empty && (!codes || !scales)) return FP4_ERR_INVALID_ARG;
+    if (!empty && double_block && !outer_scales) return FP4_ERR_INVALID_ARG;
+    if (needs_ts && !tensor_scale) return FP4_ERR_INVALID_ARG;
+    if (codes && !aligned16(codes)) return FP4_ERR_MISALIGNED;
+    if ((outer_scales && ((uintptr_t)outer_scales & 3u)) || (tensor_scale && ((uintptr_t)tensor_scale & 3u)) ||
+        (tensor_amax && ((uintptr_t)tensor_amax & 3u)))
+        return FP4_ERR_MISALIGNED;
+    if (internal_amax && !empty) {
+        if (!workspace || workspace_bytes < 256) return FP4_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    }
+    int dev;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (empty) {
+        if (needs_ts) {
+            static const float one = 1.0f;
+            if (cudaMemcpyAsync(tensor_scale, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return FP4_ERR_CUDA;
+        }
+        return FP4_OK;
+    }
+
+    QuantArgs a{};
+    a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
+    a.L = L; a.K = K;
+    a.nb4 = ((K / blk) + 3) / 4;
+    a.codes = codes; a.scales = scales; a.outer = outer_scales;
+    a.tensor_scale_out = needs_ts ? tensor_scale : nullptr;
+    a.keys = make_keys(seed);
+    a.tensor_id = tensor_id;
+    a.sign_mask = sign_mask_of(rotation, seed);
+    const int rn = rot_size(rotation);
+    const bool bf16 = in_dtype == FP4_IN_BF16;
+    if (internal_amax) {
+        if (cudaMemsetAsync(workspace, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
+        a.amax_out = static_cast<unsigned int*>(workspace);
+        if (launch_amax(a, bf16, rn, axis, s) != cudaSuccess) return FP4_ERR_CUDA;
+        a.amax_in = static_cast<const float*>(workspace);
+    } else {
+        a.amax_in = tensor_amax;
+    }
+    if (launch_quantize(a, bf16, format, rounding == FP4_SR, rn, double_block != 0, axis, s) != cudaSuccess)
+        return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
+fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
+                      const uint8_t* a_codes, const uint8_t* a_scales, const float* a_outer,
+                      const float* a_tensor_scale,
+                      const uint8_t* b_codes, const uint8_t* b_scales, const float* b_outer,
+                      const float* b_tensor_scale,
+                      int64_t M, int64_t N, int64_t K, void* c, fp4_out_dtype_t out_dtype, int64_t ldc,
+                      void* stream) {
+    if (format != FP4_MXFP4 && format != FP4_NVFP4) {
+        return format == FP4_UFP4 ? FP4_ERR_UNSUPPORTED : FP4_ERR_INVALID_ARG;
+    }
+    if (double_block != 0 && double_block != 1) return FP4_ERR_INVALID_ARG;
+    if (double_block && format != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+    if (double_block) return FP4_ERR_UNSUPPORTED;
+    if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return FP4_OK;
+    if (M % 128 || N % 128 || K % 256 || K == 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !c) return FP4_ERR_INVALID_ARG;
+    if (format == FP4_NVFP4 && !double_block && (!a_tensor_scale || !b_tensor_scale)) return FP4_ERR_INVALID_ARG;
+    if (double_block && (!a_outer || !b_outer)) return FP4_ERR_INVALID_ARG;
+    const int64_t es = out_dtype == FP4_OUT_BF16 ? 2 : 4;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
+        !aligned16(c) || (ldc * es) % 16)
+        return FP4_ERR_MISALIGNED;
+    int dev;
+    fp4_status_t st;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    GemmArgs g{};
+    g.a_codes = a_codes; g.a_scales = a_scales; g.a_outer = a_outer; g.a_ts = a_tensor_scale;
+    g.b_codes = b_codes; g.b_scales = b_scales; g.b_outer = b_outer; g.b_ts = b_tensor_scale;
+    g.M = M; g.N = N; g.K = K; g.c = c; g.ldc = ldc;
+    g.out_bf16 = out_dtype == FP4_OUT_BF16;
+    g.fmt = format;
+    g.db = double_block;
+    g.wait_limit = g_wait_limit;
+    if (launch_gemm(g, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
+fp4_status_t fp4_last_error(void* stream) {
+    int dev;
+    fp4_status_t st;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP4_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return FP4_ERR_CUDA;
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return FP4_ERR_CUDA;
+    return word ? static_cast<fp4_status_t>(word) : FP4_OK;
+}
+
+}  // extern "C"

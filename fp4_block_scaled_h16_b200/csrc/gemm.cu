@@ -1,0 +1,355 @@
+// gemm.cu -- block-scaled FP4 GEMM on the 5th-generation tensor cores of
+// sm_100a (tcgen05.mma kind::mxf4 / kind::mxf4nvf4), for the Fprop, Dgrad and
+// Wgrad GEMMs of a linear layer on FP4 operands ("Pre-addestramento di
+// Modelli Linguistici di Grandi Dimensioni con MXFP4", Metodologia; NVFP4
+// 16-groups: "TetraJet-v2" 2.A).
+//
+//   C[i, j] = alpha * sum_k qA[i, k] qB[j, k] sA[i, k / blk] sB[j, k / blk]
+//
+// Design (one CTA per SM, persistent over 128 x BN output tiles):
+//   warp 0   TMA producer: 2-D tiled loads of the packed codes (128-byte
+//            swizzle) and bulk copies of the 512-byte scale-factor atoms into
+//            a ring of STAGES shared-memory stages of 256 K-elements each;
+//   warp 1   allocates TMEM and issues, from one thread, the smem->TMEM
+//            scale-factor copies and four 128 x BN x 64 block-scaled MMAs per
+//            stage into an FP32 accumulator in TMEM;
+//   warps 2-5 epilogue: TMEM -> registers (tcgen05.ld), times alpha, convert,
+//            store to global.
+// Every mbarrier wait is bounded; a wait that runs out sets the device error
+// word to FP4_ERR_TIMEOUT, the CTA stops, lets every copy and MMA it issued
+// land, frees its TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <mutex>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fp4 {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 256;                 // K elements per stage (128 bytes of codes per row)
+constexpr int STAGES = 4;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t DRAIN_LIMIT = 1u << 22;
+constexpr unsigned int ERR_TIMEOUT = 7u;   // FP4_ERR_TIMEOUT
+
+template <int FMT, int BN>
+struct Cfg {
+    static constexpr int BLK = (FMT == MXFP4) ? 32 : 16;        // elements per scale
+    static constexpr int KB = BK / BLK;                          // scale bytes per row per stage
+    static constexpr int ATOMS = KB / 4;                         // 512-byte atoms per 128 rows
+    static constexpr uint32_t A_BYTES = BM * BK / 2;
+    static constexpr uint32_t B_BYTES = BN * BK / 2;
+    static constexpr uint32_t SFA_BYTES = BM * KB;
+    static constexpr uint32_t SFB_BYTES = BN * KB;
+    static constexpr uint32_t TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr uint32_t STAGE_BYTES = (TX + 1023) / 1024 * 1024;
+    static constexpr uint32_t SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr uint32_t SFA_COL = BN;                      // TMEM column of the A scales
+    static constexpr uint32_t SFB_COL = BN + 4 * ATOMS;          // TMEM column of the B scales
+    static constexpr uint32_t SFB_COLS_PER_ATOM = 4 * (BN / 128);
+    static_assert(SFB_COL + SFB_COLS_PER_ATOM * ATOMS <= TMEM_COLS, "TMEM budget");
+};
+
+struct GemmParams {
+    const uint8_t* a_sf;
+    const uint8_t* b_sf;
+    const float* a_ts;
+    const float* b_ts;
+    void* c;
+    int64_t ldc;
+    int M, N, K;
+    int nb4;          // scale atoms per 128 rows along K
+    int tiles_m, tiles_n;
+    uint32_t wait_limit;
+    unsigned int* err;
+};
+
+__device__ __forceinline__ void raise_timeout(const GemmParams& p, volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicExch(p.err, ERR_TIMEOUT);
+}
+
+template <int FMT, int BN, bool OUT_BF16>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const GemmParams p) {
+    using G = Cfg<FMT, BN>;
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte aligned base (the 128-byte swizzle atoms need it)
+    const uint32_t raw = sm100::smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * G::STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* drain = acc_empty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            sm100::mbar_init(&full[s], 1);
+            sm100::mbar_init(&empty[s], 1);
+        }
+        sm100::mbar_init(acc_full, 1);
+        sm100::mbar_init(acc_empty, 4);
+        sm100::mbar_init(drain, 1);
+        *abort_flag = 0;
+        sm100::fence_barrier_init();
+        sm100::prefetch_tmap(&tmA);
+        sm100::prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        sm100::tmem_alloc(tmem_slot, TMEM_COLS);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int kt_count = p.K / BK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (sm100::elect_one()) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t fills[STAGES] = {};
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN;
+                for (int kt = 0; kt < kt_count; ++kt) {
+                    if (!sm100::mbar_wait(&empty[stage], phase ^ 1u, p.wait_limit, abort_flag)) {
+                        raise_timeout(p, abort_flag);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * G::STAGE_BYTES;
+                    sm100::mbar_arrive_expect_tx(&full[stage], G::TX);
+                    sm100::tma_load_2d(st, &tmA, kt * (BK / 2), m0, &full[stage]);
+                    sm100::tma_load_2d(st + G::A_BYTES, &tmB, kt * (BK / 2), n0, &full[stage]);
+                    const int kb0 = kt * G::KB;                          // first scale column
+                    const uint8_t* sfa = p.a_sf + ((int64_t)(m0 / 128) * p.nb4 + kb0 / 4) * 512;
+                    sm100::bulk_load(st + G::A_BYTES + G::B_BYTES, sfa, G::SFA_BYTES, &full[stage]);
+#pragma unroll
+                    for (int rb = 0; rb < BN / 128; ++rb) {
+                        const uint8_t* sfb = p.b_sf + ((int64_t)(n0 / 128 + rb) * p.nb4 + kb0 / 4) * 512;
+                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES + rb * G::ATOMS * 512,
+                                         sfb, G::ATOMS * 512, &full[stage]);
+                    }
+                    fills[stage]++;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // drain: every fill issued must land before the CTA may exit
+            for (int s = 0; s < STAGES; ++s)
+                if (fills[s]) sm100::mbar_wait(&full[s], (fills[s] - 1) & 1u, DRAIN_LIMIT, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (sm100::elect_one()) {
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true, issued = false;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                if (!sm100::mbar_wait(acc_empty, acc_phase ^ 1u, p.wait_limit, abort_flag)) {
+                    raise_timeout(p, abort_flag);
+                    break;
+                }
+                sm100::tc_fence_after();
+                for (int kt = 0; kt < kt_count; ++kt) {
+                    if (!sm100::mbar_wait(&full[stage], phase, p.wait_limit, abort_flag)) {
+                        raise_timeout(p, abort_flag);
+                        ok = false;
+                        break;
+                    }
+                    sm100::tc_fence_after();
+                    const uint32_t st = sm100::smem_u32(smem + stage * G::STAGE_BYTES);
+                    const uint32_t st_sfa = st + G::A_BYTES + G::B_BYTES;
+                    const uint32_t st_sfb = st_sfa + G::SFA_BYTES;
+#pragma unroll
+                    for (int j = 0; j < G::ATOMS; ++j) {
+                        sm100::tc_cp_sf(tmem + G::SFA_COL + 4 * j, sm100::desc_sf(st_sfa + 512 * j));
+#pragma unroll
+                        for (int rb = 0; rb < BN / 128; ++rb)
+                            sm100::tc_cp_sf(tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * j + 4 * rb,
+                                            sm100::desc_sf(st_sfb + (rb * G::ATOMS + j) * 512));
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < BK / 64; ++kk) {
+                        const uint64_t da = sm100::desc_sw128(st + 32 * kk);
+                        const uint64_t db = sm100::desc_sw128(st + G::A_BYTES + 32 * kk);
+                        const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
+                        if (FMT == MXFP4) {
+                            // block 32: two scale bytes per MMA, the pair kk % 2 of atom kk / 2
+                            const int j = kk / 2;
+                            const uint32_t id = sm100::idesc_block_scaled(BN, true, (kk & 1) * 2, (kk & 1) * 2);
+                            sm100::mma_mxf4(tmem, da, db, id, tmem + G::SFA_COL + 4 * j,
+                                            tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * j, acc);
+                        } else {
+                            const uint32_t id = sm100::idesc_block_scaled(BN, false, 0, 0);
+                            sm100::mma_nvf4(tmem, da, db, id, tmem + G::SFA_COL + 4 * kk,
+                                            tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * kk, acc);
+                        }
+                    }
+                    issued = true;
+                    sm100::tc_commit(&empty[stage]);          // stage free once these MMAs are done
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                sm100::tc_commit(acc_full);                   // accumulator ready for the epilogue
+                acc_phase ^= 1u;
+            }
+            if (issued) {
+                sm100::tc_commit(drain);
+                sm100::mbar_wait(drain, 0, DRAIN_LIMIT, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        float alpha = 1.0f;
+        if (FMT == NVFP4) alpha = __fmul_rn(*p.a_ts, *p.b_ts);
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN;
+            // one lane polls, the warp follows its verdict (the TMEM loads below
+            // are warp-collective)
+            int got = 0;
+            if (lane == 0) {
+                got = sm100::mbar_wait(acc_full, acc_phase, p.wait_limit, abort_flag) ? 1 : 0;
+                if (!got) raise_timeout(p, abort_flag);
+            }
+            if (!__shfl_sync(0xffffffffu, got, 0)) break;
+            sm100::tc_fence_after();
+            const int row = m0 + 32 * q + lane;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 32 * c, r);
+                sm100::tmem_ld_wait();
+                if (OUT_BF16) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
+                                                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
+                        pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + n0 + 32 * c);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)row * p.ldc + n0 + 32 * c);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        dst[v] = make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha),
+                                             __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
+                                             __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
+                                             __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+                }
+            }
+            sm100::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(acc_empty);
+            acc_phase ^= 1u;
+        }
+    }
+
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// 2-D map over packed codes [rows, K/2] bytes, box = 128 bytes x box_rows, 128-byte swizzle
+bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT, int BN, bool OUT_BF16>
+cudaError_t run(const GemmArgs& g, cudaStream_t s) {
+    using G = Cfg<FMT, BN>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_kernel<FMT, BN, OUT_BF16>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap ta, tb;
+    if (!make_codes_map(&ta, g.a_codes, g.M, g.K, BM) || !make_codes_map(&tb, g.b_codes, g.N, g.K, BN))
+        return cudaErrorInvalidValue;
+    GemmParams p{};
+    p.a_sf = g.a_scales;
+    p.b_sf = g.b_scales;
+    p.a_ts = g.a_ts;
+    p.b_ts = g.b_ts;
+    p.c = g.c;
+    p.ldc = g.ldc;
+    p.M = (int)g.M;
+    p.N = (int)g.N;
+    p.K = (int)g.K;
+    p.nb4 = (int)(g.K / G::BLK / 4);
+    p.tiles_m = (int)(g.M / BM);
+    p.tiles_n = (int)(g.N / BN);
+    p.wait_limit = g.wait_limit;
+    p.err = device_error_word();
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    gemm_kernel<FMT, BN, OUT_BF16><<<grid, NUM_THREADS, G::SMEM, s>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
+    if (g.db) return cudaErrorNotSupported;
+    const bool n256 = (g.N % 256) == 0;
+    if (g.fmt == MXFP4) {
+        if (n256) return g.out_bf16 ? run<MXFP4, 256, true>(g, s) : run<MXFP4, 256, false>(g, s);
+        return g.out_bf16 ? run<MXFP4, 128, true>(g, s) : run<MXFP4, 128, false>(g, s);
+    }
+    if (n256) return g.out_bf16 ? run<NVFP4, 256, true>(g, s) : run<NVFP4, 256, false>(g, s);
+    return g.out_bf16 ? run<NVFP4, 128, true>(g, s) : run<NVFP4, 128, false>(g, s);
+}
+
+}  // namespace fp4

@@ -1,0 +1,55 @@
+// internal.h -- declarations shared by the CUDA translation units of libfp4.so.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp4_device.cuh"
+
+namespace fp4 {
+
+// arguments of the quantizer and amax kernels (passed by value)
+struct QuantArgs {
+    const void* x;
+    int64_t rows, cols, ld;     // input [rows, ld], `cols` valid columns
+    int64_t L, K, nb4;          // lines, elements per line, ceil((K / block) / 4)
+    uint8_t* codes;
+    uint8_t* scales;
+    float* outer;
+    float* tensor_scale_out;
+    const float* amax_in;       // rotated-tensor amax (NVFP4 / UFP4 without double block)
+    unsigned int* amax_out;     // amax pass: atomicMax target (binary32 bits, >= 0)
+    PhiloxKeys keys;
+    uint32_t tensor_id;
+    uint32_t sign_mask;         // random-sign bits (0: deterministic Hadamard)
+};
+
+cudaError_t launch_quantize(const QuantArgs& a, bool bf16, int fmt, bool sr, int rot_n, bool db,
+                            int axis, cudaStream_t s);
+cudaError_t launch_amax(const QuantArgs& a, bool bf16, int rot_n, int axis, cudaStream_t s);
+
+// GEMM
+struct GemmArgs {
+    const uint8_t* a_codes;
+    const uint8_t* a_scales;
+    const float* a_outer;
+    const float* a_ts;
+    const uint8_t* b_codes;
+    const uint8_t* b_scales;
+    const float* b_outer;
+    const float* b_ts;
+    int64_t M, N, K;
+    void* c;
+    int64_t ldc;
+    int out_bf16;
+    int fmt;
+    int db;
+    uint32_t wait_limit;
+};
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// device state
+int num_sms();
+unsigned int* device_error_word();   // device address of the error word of the current device
+
+}  // namespace fp4

@@ -1,0 +1,181 @@
+"""ctypes binding of libfp4.so (C ABI in include/fp4.h).
+
+Argument marshalling only: every step of quantization and GEMM runs in the
+library's CUDA kernels.  Pointer arguments take a torch tensor (its
+``data_ptr()``), an integer address or None; ``stream`` defaults to torch's
+current CUDA stream.  A non-OK status raises :class:`Fp4Error`.
+
+Importing this module loads the library and raises ImportError if it has not
+been built (``python -m fp4_block_scaled_h16_b200.build``): there is no CPU
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp4.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libfp4.so is not built: run `python -m fp4_block_scaled_h16_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# enums (include/fp4.h)
+FP4_OK, FP4_ERR_INVALID_ARG, FP4_ERR_UNSUPPORTED_SHAPE, FP4_ERR_MISALIGNED = 0, 1, 2, 3
+FP4_ERR_WORKSPACE, FP4_ERR_NO_DEVICE, FP4_ERR_CUDA, FP4_ERR_TIMEOUT, FP4_ERR_UNSUPPORTED = 4, 5, 6, 7, 8
+FP4_MXFP4, FP4_NVFP4, FP4_UFP4 = 0, 1, 2
+FP4_RTNE, FP4_SR = 0, 1
+FP4_ROT_NONE, FP4_ROT_H16, FP4_ROT_H32, FP4_ROT_RH16, FP4_ROT_RH32 = 0, 1, 2, 3, 4
+FP4_IN_F32, FP4_IN_BF16 = 0, 1
+FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
+
+EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_quantize",
+           "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit")
+
+_P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
+                                 ctypes.c_uint32, ctypes.c_size_t)
+_lib.fp4_status_string.argtypes = [_I]
+_lib.fp4_status_string.restype = ctypes.c_char_p
+_lib.fp4_scales_bytes.argtypes = [_I64, _I64, _I]
+_lib.fp4_scales_bytes.restype = _SZ
+_lib.fp4_quantize_workspace_size.argtypes = [_I, _I, _I, ctypes.POINTER(_SZ)]
+_lib.fp4_amax.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _P, _P]
+_lib.fp4_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _I, _U64, _U32, _P,
+                              _P, _P, _P, _P, _P, _SZ, _P]
+_lib.fp4_gemm.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P]
+_lib.fp4_last_error.argtypes = [_P]
+_lib.fp4_set_wait_limit.argtypes = [_U32]
+_lib.fp4_set_wait_limit.restype = None
+for _f in ("fp4_amax", "fp4_quantize", "fp4_gemm", "fp4_last_error", "fp4_quantize_workspace_size"):
+    getattr(_lib, _f).restype = _I
+
+
+class Fp4Error(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        super().__init__("%s%s" % (where + ": " if where else "", fp4_status_string(status)))
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != FP4_OK:
+        raise Fp4Error(status, where)
+
+
+def fp4_status_string(status: int) -> str:
+    return _lib.fp4_status_string(status).decode()
+
+
+def fp4_scales_bytes(lines: int, K: int, fmt: int) -> int:
+    return _lib.fp4_scales_bytes(lines, K, fmt)
+
+
+def fp4_quantize_workspace_size(fmt: int, double_block: bool, amax_given: bool) -> int:
+    n = _SZ(0)
+    _check(_lib.fp4_quantize_workspace_size(fmt, int(double_block), int(amax_given), ctypes.byref(n)),
+           "fp4_quantize_workspace_size")
+    return n.value
+
+
+def fp4_set_wait_limit(polls: int) -> None:
+    _lib.fp4_set_wait_limit(polls)
+
+
+def fp4_amax(x, in_dtype, rows, cols, ld, rotation, axis, seed, amax_out, stream=None) -> None:
+    _check(_lib.fp4_amax(_ptr(x), in_dtype, rows, cols, ld, rotation, axis, seed, _ptr(amax_out),
+                         _stream(stream)), "fp4_amax")
+
+
+def fp4_quantize(x, in_dtype, rows, cols, ld, fmt, rounding, rotation, axis, double_block, seed,
+                 tensor_id, tensor_amax, codes, scales, outer_scales, tensor_scale, workspace,
+                 workspace_bytes, stream=None) -> None:
+    _check(_lib.fp4_quantize(_ptr(x), in_dtype, rows, cols, ld, fmt, rounding, rotation, axis,
+                             int(double_block), seed, tensor_id, _ptr(tensor_amax), _ptr(codes),
+                             _ptr(scales), _ptr(outer_scales), _ptr(tensor_scale), _ptr(workspace),
+                             workspace_bytes, _stream(stream)), "fp4_quantize")
+
+
+def fp4_gemm(fmt, double_block, a_codes, a_scales, a_outer, a_tensor_scale, b_codes, b_scales,
+             b_outer, b_tensor_scale, M, N, K, c, out_dtype, ldc, stream=None) -> None:
+    _check(_lib.fp4_gemm(fmt, int(double_block), _ptr(a_codes), _ptr(a_scales), _ptr(a_outer),
+                         _ptr(a_tensor_scale), _ptr(b_codes), _ptr(b_scales), _ptr(b_outer),
+                         _ptr(b_tensor_scale), M, N, K, _ptr(c), out_dtype, ldc, _stream(stream)),
+           "fp4_gemm")
+
+
+def fp4_last_error(stream=None) -> int:
+    """Status of the device error word (FP4_OK or FP4_ERR_TIMEOUT); clears it."""
+    return _lib.fp4_last_error(_stream(stream))
+
+
+# --------------------------------------------------------------------------- helpers
+# Device buffers for a quantized tensor, allocated with torch (plumbing only).
+
+def in_dtype_of(x) -> int:
+    import torch
+    if x.dtype == torch.bfloat16:
+        return FP4_IN_BF16
+    if x.dtype == torch.float32:
+        return FP4_IN_F32
+    raise TypeError("input must be bfloat16 or float32, got %s" % x.dtype)
+
+
+def alloc_qtensor(lines: int, K: int, fmt: int, double_block: bool = False, device="cuda"):
+    """codes [L, K/2] u8, tiled scales, outer [L, K/128] f32 (double block), tensor scale f32."""
+    import torch
+    return dict(
+        codes=torch.empty((lines, K // 2), dtype=torch.uint8, device=device),
+        scales=torch.empty(max(fp4_scales_bytes(lines, K, fmt), 16), dtype=torch.uint8, device=device),
+        outer=torch.empty((lines, max(K // 128, 1)), dtype=torch.float32, device=device) if double_block else None,
+        tensor_scale=torch.empty(1, dtype=torch.float32, device=device),
+        lines=lines, K=K, format=fmt, double_block=bool(double_block))
+
+
+def quantize(x, fmt, rounding=FP4_RTNE, rotation=FP4_ROT_NONE, axis=1, double_block=False, seed=0,
+             tensor_id=0, tensor_amax=None, out=None, workspace=None, cols=None, stream=None):
+    """Quantize a 2-D CUDA tensor (row-major, unit stride in the last dim) into a new or given qtensor."""
+    import torch
+    rows, ld = x.shape[0], x.stride(0) if x.dim() == 2 and x.shape[0] > 1 else x.shape[1]
+    cols = x.shape[1] if cols is None else cols
+    K, L = (cols, rows) if axis == 1 else (rows, cols)
+    q = out if out is not None else alloc_qtensor(L, K, fmt, double_block, x.device)
+    ws_bytes = fp4_quantize_workspace_size(fmt, double_block, tensor_amax is not None)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+    fp4_quantize(x, in_dtype_of(x), rows, cols, ld, fmt, rounding, rotation, axis, double_block, seed,
+                 tensor_id, tensor_amax, q["codes"], q["scales"], q["outer"], q["tensor_scale"],
+                 workspace if ws_bytes else None, ws_bytes, stream)
+    return q
+
+
+def gemm(qa, qb, out_dtype=FP4_OUT_F32, out=None, stream=None):
+    """C = A B^T on two quantized tensors of the same format (lines along K)."""
+    import torch
+    M, N, K = qa["lines"], qb["lines"], qa["K"]
+    if qb["K"] != K or qa["format"] != qb["format"] or qa["double_block"] != qb["double_block"]:
+        raise ValueError("operands must share K, format and double-block mode")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16 if out_dtype == FP4_OUT_BF16 else torch.float32,
+                          device=qa["codes"].device)
+    fp4_gemm(qa["format"], qa["double_block"], qa["codes"], qa["scales"], qa["outer"], qa["tensor_scale"],
+             qb["codes"], qb["scales"], qb["outer"], qb["tensor_scale"], M, N, K, out, out_dtype,
+             out.stride(0), stream)
+    return out

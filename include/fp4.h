@@ -1,0 +1,225 @@
+/*
+ * fp4.h -- C ABI of libfp4.so: block-scaled FP4 quantization and block-scaled
+ * FP4 GEMMs on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources are page titles and sections):
+ *   - "Pre-addestramento di Modelli Linguistici di Grandi Dimensioni con MXFP4",
+ *     Metodologia: MXFP4 on the Fprop, Dgrad and Wgrad GEMMs of every linear
+ *     layer, stabilised by deterministic 16x16 / 32x32 Hadamard rotations
+ *     (H16 / H32), with stochastic rounding and randomised Hadamard as the
+ *     alternatives studied.
+ *   - "Ripensare il Bias di Shrinkage nel Pretraining di LLM in FP4",
+ *     Problematica and Metodologia 1-2: the E2M1 grid under round-to-nearest-
+ *     even, the uniform UFP4 grid (levels k*s, k in [-7, 7]), random Hadamard
+ *     on all three GEMMs, stochastic rounding on the upstream gradient.
+ *   - "TetraJet-v2", section 2.A: NVFP4 = E2M1 in 16-element groups with an
+ *     8-bit (E4M3) scale; the double-block variant, a 128-element outer block
+ *     with an FP32 scale over 16-element inner blocks; stochastic rounding in
+ *     the backward pass; 1x16 weight groups re-quantized along the transposed
+ *     axis for the backward GEMMs.
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers of the current CUDA device, owned
+ *     and allocated by the caller; the library allocates no memory and keeps
+ *     no per-call state.
+ *   - `stream` is a cudaStream_t passed as void* (NULL: the legacy default
+ *     stream).  Calls are asynchronous on it: outputs are valid once the
+ *     stream has reached the call.
+ *   - Argument, shape and alignment errors are returned synchronously and
+ *     nothing is launched.  A failed launch returns FP4_ERR_CUDA.  Device-side
+ *     timeouts of the GEMM pipeline are reported by fp4_last_error().
+ *   - Pointers to tensor data must be 16-byte aligned.
+ *
+ * Quantized tensor ("K-major view")
+ *   A quantized tensor has L lines of K elements each, quantized along the
+ *   line.  For axis = 1 the lines are the rows of the [R, C] input (L = R,
+ *   K = C); for axis = 0 they are its columns (L = C, K = R), so the output is
+ *   the transposed tensor, as the Dgrad / Wgrad operands need.
+ *     codes   uint8 [L, K/2]: 4-bit codes, element 2j in the low nibble of
+ *             byte j.  Code = sign << 3 | magnitude index; E2M1 magnitudes
+ *             {0, .5, 1, 1.5, 2, 3, 4, 6}, UFP4 magnitudes k = 0..7.
+ *     scales  one byte per block of the line (block 32 for MXFP4: E8M0, value
+ *             2^(byte - 127); block 16 for NVFP4/UFP4: E4M3), in the tiled
+ *             layout below.
+ *     outer   float [L, K/128] row-major (double block only).
+ *     tensor_scale  one float (NVFP4/UFP4 without double block).
+ *   Element value = q * s_block (MXFP4), q * s_block * tensor_scale (NVFP4,
+ *   UFP4), q * s_block * outer[l][k/128] (double block).
+ *
+ * Tiled scale layout (the layout the tcgen05 block-scaled MMA reads): with
+ * nb = K / block scale bytes per line, the byte of line l, block b is at
+ *     ((l / 128) * ceil(nb / 4) + b / 4) * 512
+ *       + (l % 32) * 16 + ((l % 128) / 32) * 4 + (b % 4)
+ * and the buffer holds fp4_scales_bytes(L, K, format) bytes (L rounded up to
+ * 128 and nb to 4).  Padding bytes are never written.
+ */
+#ifndef FP4_H
+#define FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP4_OK = 0,
+    FP4_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size */
+    FP4_ERR_UNSUPPORTED_SHAPE = 2, /* a size breaks the shape rules */
+    FP4_ERR_MISALIGNED = 3,        /* a pointer or leading dimension is not 16-byte aligned */
+    FP4_ERR_WORKSPACE = 4,         /* workspace missing or too small */
+    FP4_ERR_NO_DEVICE = 5,         /* no CUDA device, or not a B200-class (sm_100) device */
+    FP4_ERR_CUDA = 6,              /* a CUDA runtime call failed */
+    FP4_ERR_TIMEOUT = 7,           /* a device-side wait gave up (reported by fp4_last_error) */
+    FP4_ERR_UNSUPPORTED = 8        /* a valid combination this build does not implement */
+} fp4_status_t;
+
+typedef enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1, FP4_UFP4 = 2 } fp4_format_t;
+typedef enum { FP4_RTNE = 0, FP4_SR = 1 } fp4_rounding_t;
+typedef enum {
+    FP4_ROT_NONE = 0,
+    FP4_ROT_H16 = 1,   /* deterministic 16x16 Sylvester Hadamard, scaled by 1/4 */
+    FP4_ROT_H32 = 2,   /* deterministic 32x32, scaled by binary32(1/sqrt(32)) */
+    FP4_ROT_RH16 = 3,  /* random signs then H16 */
+    FP4_ROT_RH32 = 4   /* random signs then H32 */
+} fp4_rotation_t;
+typedef enum { FP4_IN_F32 = 0, FP4_IN_BF16 = 1 } fp4_in_dtype_t;
+typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype_t;
+
+/*
+ * fp4_scales_bytes -- size in bytes of the tiled scale buffer of a quantized
+ * tensor with `lines` lines of K elements in `format` (0 for an empty tensor).
+ */
+size_t fp4_scales_bytes(int64_t lines, int64_t K, fp4_format_t format);
+
+/*
+ * fp4_quantize_workspace_size -- device workspace fp4_quantize needs for this
+ * format / amax choice: 256 bytes when the tensor amax is computed internally
+ * (NVFP4 or UFP4, no double block, tensor_amax == NULL), otherwise 0.
+ * Returns FP4_ERR_INVALID_ARG for a bad format or a null `bytes`.
+ */
+fp4_status_t fp4_quantize_workspace_size(fp4_format_t format, int double_block,
+                                         int amax_given, size_t* bytes);
+
+/*
+ * fp4_amax -- amax of the rotated tensor: max |y| over all elements, where y
+ * is x rotated on every aligned n-block along the quantization axis (no
+ * rotation: max |x|).  This is the amax the NVFP4 / UFP4 tensor scale
+ * amax / (Q * 448) is taken from ("TetraJet-v2" 2.A: the tensor-wide amax that
+ * the double block avoids); calling it separately lets a caller combine the
+ * amax of several shards (a max all-reduce) before quantizing each shard.
+ *
+ *   x         device, [rows, ld] row-major, `cols` <= ld valid columns
+ *   rotation  rotation along the axis; its size must divide the axis length
+ *   seed      selects the random signs of FP4_ROT_RH16 / RH32
+ *   amax_out  device, one float, overwritten
+ * Empty input (rows or cols == 0) writes 0.
+ */
+fp4_status_t fp4_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols,
+                      int64_t ld, fp4_rotation_t rotation, int axis, uint64_t seed,
+                      float* amax_out, void* stream);
+
+/*
+ * fp4_quantize -- fused rotate / amax / scale / round / pack of one tensor.
+ *
+ * Steps, on every line of K elements along `axis`:
+ *   1. load and widen to binary32 (bf16 -> f32 is exact);
+ *   2. rotation (optional): x <- d . x (random signs: bit j of word 0 of
+ *      Philox4x32-10(key = seed, counter = (0, 0, 0, 1)), set = -1), then the
+ *      Sylvester butterfly in binary32 for h = 1, 2, ..., n/2, then times
+ *      c_n (c_16 = 0.25, c_32 = binary32(1/sqrt 32));
+ *   3. scale per block, with m the block amax:
+ *      MXFP4 (block 32): e = clamp(floor(log2 m) - 2, -127, 127) (m = 0:
+ *        -127), byte e + 127, v = x * 2^-e;
+ *      NVFP4 / UFP4 (block 16, Q = 6 / 7): s_t = A / (Q * 448) from the
+ *        tensor amax A (1 if A = 0), s_b = E4M3_rne_satfinite((m / Q) / s_t),
+ *        v = x / (s_b * s_t); s_b = 0 gives signed zero codes;
+ *      double block (NVFP4 only): s_o = m128 / 2688 per 128-element chunk of
+ *        the line (1 if m128 = 0) replaces s_t;
+ *   4. round |v| onto the grid (clamped to the top level), sign from x:
+ *      FP4_RTNE: nearest, ties to the even magnitude index;
+ *      FP4_SR: up from the level below with probability (|v| - lo)/(hi - lo),
+ *        using word (i mod 4) of Philox4x32-10(key = seed, counter =
+ *        (lo32(i/4), hi32(i/4), tensor_id, 0)) for input element (r, c),
+ *        i = r * cols + c: up iff (word >> 8) * 2^-24 < (|v| - lo)/(hi - lo);
+ *   5. pack two codes per byte and store codes and scales.
+ *
+ * Arguments
+ *   x, in_dtype, rows, cols, ld   input [rows, ld] row-major, `cols` valid
+ *                                 columns; ld * sizeof(element) % 16 == 0
+ *   format, rounding, rotation    as above
+ *   axis            1: lines are rows (K = cols); 0: lines are columns
+ *                   (K = rows), i.e. the transposed tensor is written
+ *   double_block    NVFP4 only: FP32 outer scale per 128 elements
+ *   seed, tensor_id SR stream and random signs (tensor_id only for SR)
+ *   tensor_amax     optional device float: the rotated-tensor amax to build
+ *                   s_t from (e.g. the max over shards); NULL = computed here,
+ *                   which needs the workspace
+ *   codes           device uint8 [L, K/2]
+ *   scales          device, fp4_scales_bytes(L, K, format) bytes, tiled layout
+ *   outer_scales    device float [L, K/128] (double block), else ignored
+ *   tensor_scale    device float, receives s_t (NVFP4/UFP4, no double block)
+ *   workspace       device, >= fp4_quantize_workspace_size() bytes, 16-byte
+ *                   aligned; contents are scratch
+ * Shape rules: K % block == 0 (32 MXFP4, 16 NVFP4/UFP4), K % n == 0 for a
+ * rotation of size n, K % 128 == 0 for double block; L may be anything >= 0.
+ */
+fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols,
+                          int64_t ld, fp4_format_t format, fp4_rounding_t rounding,
+                          fp4_rotation_t rotation, int axis, int double_block,
+                          uint64_t seed, uint32_t tensor_id, const float* tensor_amax,
+                          uint8_t* codes, uint8_t* scales, float* outer_scales,
+                          float* tensor_scale, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
+ * fp4_gemm -- block-scaled FP4 GEMM on tcgen05 tensor cores:
+ *     C[i, j] = alpha_ij * sum_k qA[i, k] qB[j, k] sA[i, k/blk] sB[j, k/blk]
+ * with A [M, K] and B [N, K] quantized tensors in the K-major view (lines
+ * along K) of the same format, as fp4_quantize writes them:
+ *   MXFP4:  alpha = 1, blk = 32 (E8M0 scales);
+ *   NVFP4:  alpha = a_tensor_scale * b_tensor_scale, blk = 16 (E4M3);
+ *   double block: alpha varies per 128-element K chunk:
+ *           a_outer[i, k/128] * b_outer[j, k/128].
+ * This is the Fprop (Y = X W^T), Dgrad (dX = dY W: B = W quantized on
+ * axis 0) and Wgrad (dW = dY^T X: both quantized on axis 0) GEMM of a linear
+ * layer ("Pre-addestramento ... con MXFP4", Metodologia).  Rotations cancel
+ * in the contraction only if both operands used the same rotation and seed;
+ * the GEMM applies no inverse rotation.
+ *
+ *   c         device, [M, ldc] row-major, fp32 or bf16, ldc >= N
+ * Shape rules: M % 128 == 0, N % 128 == 0, K % 256 == 0; ldc * size % 16 == 0.
+ * The accumulation is FP32 on the tensor cores.
+ */
+fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
+                      const uint8_t* a_codes, const uint8_t* a_scales,
+                      const float* a_outer, const float* a_tensor_scale,
+                      const uint8_t* b_codes, const uint8_t* b_scales,
+                      const float* b_outer, const float* b_tensor_scale,
+                      int64_t M, int64_t N, int64_t K,
+                      void* c, fp4_out_dtype_t out_dtype, int64_t ldc, void* stream);
+
+/*
+ * fp4_last_error -- synchronizes `stream` and returns (and clears) the device
+ * error word the kernels set: FP4_ERR_TIMEOUT when a bounded wait in the GEMM
+ * pipeline gave up (the kernel then abandons its tile and exits cleanly),
+ * FP4_OK otherwise, FP4_ERR_CUDA if the synchronization failed.
+ */
+fp4_status_t fp4_last_error(void* stream);
+
+/* fp4_status_string -- a static, human-readable name of a status code. */
+const char* fp4_status_string(fp4_status_t status);
+
+/*
+ * fp4_set_wait_limit -- iteration limit of every bounded device-side wait
+ * (default 2^20 polls, far above any legitimate wait).  A test can lower it to
+ * make a wait run out without hanging the GPU.  0 restores the default.
+ */
+void fp4_set_wait_limit(uint32_t polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4_H */

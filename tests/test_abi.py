@@ -1,0 +1,108 @@
+"""The C ABI library loads, exports every entry point include/fp4.h declares,
+and validates arguments on the host (no GPU needed, nothing launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp4.h")
+
+fp4 = pytest.importorskip("fp4_block_scaled_h16_b200.fp4", reason="libfp4.so not built")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 8
+    lib = ctypes.CDLL(fp4.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(fp4.EXPORTS)
+
+
+def test_status_strings():
+    assert fp4.fp4_status_string(0) == "FP4_OK"
+    assert fp4.fp4_status_string(7) == "FP4_ERR_TIMEOUT"
+    assert fp4.fp4_status_string(99) == "FP4_ERR_UNKNOWN"
+
+
+def test_scales_bytes_and_workspace():
+    assert fp4.fp4_scales_bytes(0, 64, fp4.FP4_NVFP4) == 0
+    assert fp4.fp4_scales_bytes(1, 16, fp4.FP4_NVFP4) == 128 * 4
+    assert fp4.fp4_scales_bytes(129, 4096, fp4.FP4_NVFP4) == 256 * 256
+    assert fp4.fp4_scales_bytes(256, 512, fp4.FP4_MXFP4) == 256 * 16
+    assert fp4.fp4_quantize_workspace_size(fp4.FP4_NVFP4, False, False) == 256
+    assert fp4.fp4_quantize_workspace_size(fp4.FP4_NVFP4, False, True) == 0
+    assert fp4.fp4_quantize_workspace_size(fp4.FP4_NVFP4, True, False) == 0
+    assert fp4.fp4_quantize_workspace_size(fp4.FP4_MXFP4, False, False) == 0
+    with pytest.raises(fp4.Fp4Error):
+        fp4.fp4_quantize_workspace_size(7, False, False)
+
+
+ADDR = 1 << 20       # a fake, 16-byte aligned address: validation fails before any use
+
+
+def q(**kw):
+    args = dict(x=ADDR, in_dtype=fp4.FP4_IN_BF16, rows=256, cols=512, ld=512, fmt=fp4.FP4_NVFP4,
+                rounding=fp4.FP4_RTNE, rotation=fp4.FP4_ROT_H16, axis=1, double_block=0, seed=0,
+                tensor_id=0, tensor_amax=None, codes=ADDR, scales=ADDR, outer_scales=None,
+                tensor_scale=ADDR, workspace=ADDR, workspace_bytes=256)
+    args.update(kw)
+    return fp4._lib.fp4_quantize(args["x"], args["in_dtype"], args["rows"], args["cols"], args["ld"],
+                                 args["fmt"], args["rounding"], args["rotation"], args["axis"],
+                                 args["double_block"], args["seed"], args["tensor_id"], args["tensor_amax"],
+                                 args["codes"], args["scales"], args["outer_scales"], args["tensor_scale"],
+                                 args["workspace"], args["workspace_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(in_dtype=5), 1), (dict(fmt=3), 1), (dict(rounding=2), 1), (dict(rotation=9), 1),
+    (dict(axis=2), 1), (dict(rows=-1), 1), (dict(ld=100), 1), (dict(x=None), 1),
+    (dict(codes=None), 1), (dict(tensor_scale=None), 1), (dict(double_block=1, fmt=fp4.FP4_MXFP4), 1),
+    (dict(double_block=1, outer_scales=None), 1),
+    (dict(x=ADDR + 8), 3), (dict(ld=516, cols=512), 3), (dict(codes=ADDR + 4), 3),
+    (dict(cols=500, ld=512), 2), (dict(fmt=fp4.FP4_MXFP4, cols=496, ld=512), 2),
+    (dict(rotation=fp4.FP4_ROT_H32, cols=496, ld=512), 2),
+    (dict(double_block=1, outer_scales=ADDR, cols=448, ld=448), 2),
+    (dict(axis=0, rows=200), 2),
+    (dict(workspace=None), 4), (dict(workspace_bytes=16), 4),
+])
+def test_quantize_host_validation(kw, status):
+    assert q(**kw) == status
+
+
+def g(**kw):
+    args = dict(fmt=fp4.FP4_NVFP4, db=0, a=ADDR, sa=ADDR, oa=None, ta=ADDR, b=ADDR, sb=ADDR, ob=None, tb=ADDR,
+                M=256, N=256, K=512, c=ADDR, out=fp4.FP4_OUT_BF16, ldc=256)
+    args.update(kw)
+    return fp4._lib.fp4_gemm(args["fmt"], args["db"], args["a"], args["sa"], args["oa"], args["ta"], args["b"],
+                             args["sb"], args["ob"], args["tb"], args["M"], args["N"], args["K"], args["c"],
+                             args["out"], args["ldc"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(fmt=7), 1), (dict(fmt=fp4.FP4_UFP4), 8), (dict(out=3), 1), (dict(ldc=100), 1),
+    (dict(M=-128), 1), (dict(a=None), 1), (dict(ta=None), 1), (dict(db=1, fmt=fp4.FP4_MXFP4), 1),
+    (dict(M=200), 2), (dict(N=192), 2), (dict(K=384), 2), (dict(K=0), 2),
+    (dict(a=ADDR + 8), 3), (dict(ldc=260), 3),
+])
+def test_gemm_host_validation(kw, status):
+    assert g(**kw) == status
+
+
+def test_empty_gemm_is_a_no_op():
+    assert g(M=0) == 0 and g(N=0, ldc=0) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
+def test_valid_call_without_gpu_reports_no_device():
+    assert q() == fp4.FP4_ERR_NO_DEVICE
+    assert g() == fp4.FP4_ERR_NO_DEVICE

@@ -1,0 +1,133 @@
+"""GEMM parity: the tcgen05 block-scaled FP4 GEMM (through the C ABI) against
+the oracle's float64 GEMM of the exactly dequantized operands, per element
+within |C - C64| <= 1e-5 * sum_k |a_ik b_jk| (plus half a bf16 ulp of the
+result for bf16 output).
+
+Operands: first the oracle's own quantized tensors uploaded to the GPU (the
+GEMM alone), then the whole path (GPU quantizer -> GPU GEMM against oracle
+quantizer -> oracle GEMM), at small sizes in full and at the full
+Llama-3.1-8B-shaped sizes on sampled rows and columns.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import (assert_quant_equal, assert_within_gemm_bound, gpu_quantize, oracle_quantize,
+                    sample_lines, upload_oracle_qtensor)
+from fp4_block_scaled_h16_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+MX, NV = 0, 1
+
+
+@pytest.fixture(scope="module")
+def fp4(cuda_device):
+    from fp4_block_scaled_h16_b200 import fp4 as m
+    return m
+
+
+def rand(M, K, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((M, K)) * scale).astype(np.float32)
+    x[:, rng.choice(K, 2, replace=False)] *= 30.0
+    return torch.from_numpy(x)
+
+
+@pytest.mark.parametrize("out_bf16", [False, True])
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 512), (384, 256, 1024), (128, 512, 2304)])
+def test_gemm_on_oracle_operands(fp4, fmt, out_bf16, shape):
+    M, N, K = shape
+    a, b = rand(M, K, M + K + fmt), rand(N, K, N + 3 * K + fmt, 0.1)
+    qa = oracle_quantize(a, fmt=fmt, rotation=1)
+    qb = oracle_quantize(b, fmt=fmt, rotation=1)
+    C64, bound = oracle.gemm(qa, qb)
+    ta, tb = upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb)
+    C = fp4.gemm(ta, tb, fp4.FP4_OUT_BF16 if out_bf16 else fp4.FP4_OUT_F32)
+    torch.cuda.synchronize()
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    assert_within_gemm_bound(C.float().cpu().numpy(), C64, bound, out_bf16, what=str((fmt, shape, out_bf16)))
+
+
+def test_gemm_ldc_larger_than_n(fp4):
+    a, b = rand(128, 512, 1), rand(256, 512, 2)
+    qa, qb = oracle_quantize(a, fmt=NV), oracle_quantize(b, fmt=NV)
+    C64, bound = oracle.gemm(qa, qb)
+    out = torch.full((128, 264), 7.0, dtype=torch.float32, device="cuda")
+    fp4.gemm(upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb), fp4.FP4_OUT_F32,
+             out=out[:, :256])
+    torch.cuda.synchronize()
+    o = out.cpu().numpy()
+    assert (o[:, 256:] == 7.0).all()
+    assert_within_gemm_bound(o[:, :256], C64, bound, False)
+
+
+def test_gemm_zero_and_extreme_scales(fp4):
+    a = torch.zeros((128, 512))
+    a[3, :] = 1e30
+    a[5, :] = 1e-30
+    b = rand(128, 512, 9)
+    for fmt in (MX, NV):
+        qa, qb = oracle_quantize(a, fmt=fmt), oracle_quantize(b, fmt=fmt)
+        C64, bound = oracle.gemm(qa, qb)
+        C = fp4.gemm(upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb), fp4.FP4_OUT_F32)
+        torch.cuda.synchronize()
+        assert_within_gemm_bound(C.cpu().numpy(), C64, bound, False)
+
+
+def test_tiny_mxfp4_end_to_end(fp4):
+    """A fp32 256x512 (axis 1) times B fp32 512x256 (axis 0): C = A B, fp32 out."""
+    d = workloads.tiny_mxfp4()
+    ga = gpu_quantize(fp4, d["A"].cuda(), fmt=MX, axis=1)
+    gb = gpu_quantize(fp4, d["B"].cuda(), fmt=MX, axis=0)
+    oa, ob = oracle_quantize(d["A"], fmt=MX, axis=1), oracle_quantize(d["B"], fmt=MX, axis=0)
+    assert_quant_equal(ga, oa)
+    assert_quant_equal(gb, ob)
+    C = fp4.gemm(ga["raw"], gb["raw"], fp4.FP4_OUT_F32)
+    torch.cuda.synchronize()
+    C64, bound = oracle.gemm(oa, ob)
+    assert_within_gemm_bound(C.cpu().numpy(), C64, bound, False, what="tiny")
+    # the quantized product is close to the exact one
+    ref = d["A"].double().numpy() @ d["B"].double().numpy()
+    assert np.abs(C.cpu().numpy() - ref).max() < 0.25 * np.abs(ref).max()
+
+
+def sampled_gemm_check(fp4, qa_dev, qb_dev, x_a, x_b, kw_a, kw_b, out_bf16, n, seed):
+    C = fp4.gemm(qa_dev, qb_dev, fp4.FP4_OUT_BF16 if out_bf16 else fp4.FP4_OUT_F32)
+    torch.cuda.synchronize()
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    rows = sample_lines(qa_dev["lines"], n, seed)
+    cols = sample_lines(qb_dev["lines"], n, seed + 1)
+    oa = oracle_quantize(x_a, lines=rows, **kw_a)
+    ob = oracle_quantize(x_b, lines=cols, **kw_b)
+    C64, bound = oracle.gemm(oa, ob)
+    sub = C.float()[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].cpu().numpy()
+    return assert_within_gemm_bound(sub, C64, bound, out_bf16)
+
+
+def test_full_nvfp4_fprop_qkv(fp4):
+    """Y = X W^T, X 8192x4096, W 6144x4096, NVFP4 + H16, bf16 out 8192x6144."""
+    d = workloads.nvfp4_fprop_qkv()
+    kw = dict(fmt=NV, rounding=0, rotation=1, axis=1)
+    qx = fp4.quantize(d["X"].cuda(), **kw)
+    qw = fp4.quantize(d["W"].cuda(), **kw)
+    sampled_gemm_check(fp4, qx, qw, d["X"], d["W"], kw, kw, True, 128, 0)
+
+
+def test_full_mxfp4_wgrad_down(fp4):
+    """dW = dY^T H: both quantized along the 8192 tokens, random-sign H32, SR; fp32 out 4096x14336."""
+    d = workloads.mxfp4_wgrad_down()
+    ka = dict(fmt=MX, rounding=1, rotation=4, axis=0, seed=0, tensor_id=1)
+    kb = dict(fmt=MX, rounding=1, rotation=4, axis=0, seed=0, tensor_id=2)
+    qa = fp4.quantize(d["dY"].cuda(), **ka)
+    qb = fp4.quantize(d["H"].cuda(), **kb)
+    sampled_gemm_check(fp4, qa, qb, d["dY"], d["H"], ka, kb, False, 96, 1)
+
+
+def test_double_block_gemm_not_yet(fp4):
+    a = rand(128, 512, 1)
+    qa = fp4.quantize(a.cuda(), fmt=NV, double_block=True)
+    with pytest.raises(fp4.Fp4Error) as e:
+        fp4.gemm(qa, qa)
+    assert e.value.status == fp4.FP4_ERR_UNSUPPORTED
