@@ -176,9 +176,12 @@ __device__ __forceinline__ uint32_t nv_scale(float* v, float m, float s_ref, boo
     return E;
 }
 
+// amax / (Q * 448); 1 when that is 0 (amax 0, or an amax so small the
+// quotient underflows), as for an all-zero block
 __device__ __forceinline__ float tensor_scale_of(float amax, int fmt) {
     const float q448 = (fmt == UFP4) ? 3136.0f : 2688.0f;
-    return amax > 0.0f ? __fdiv_rn(amax, q448) : 1.0f;
+    const float s = __fdiv_rn(amax, q448);
+    return s > 0.0f ? s : 1.0f;
 }
 
 // -------------------------------------------------------------------- axis = 1 kernel
@@ -242,7 +245,7 @@ quant_rows_kernel(const QuantArgs a) {
                 float m = absmax(v, U);
 #pragma unroll
                 for (int s = 1; s < G; s <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, s));
-                s_ref = m > 0.0f ? __fdiv_rn(m, 2688.0f) : 1.0f;
+                s_ref = tensor_scale_of(m, NVFP4);
                 if (active && (lane & (G - 1)) == 0)
                     a.outer[l * (a.K / 128) + (j * U) / 128] = s_ref;
             }
@@ -364,7 +367,7 @@ quant_cols_kernel(const QuantArgs a) {
         for (int cc = 0; cc < 2; ++cc) {
             const int c = 2 * lane + cc;
             const float m = fmaxf(fmaxf(chunk_max[0][c], chunk_max[1][c]), fmaxf(chunk_max[2][c], chunk_max[3][c]));
-            s_ref[cc] = m > 0.0f ? __fdiv_rn(m, 2688.0f) : 1.0f;
+            s_ref[cc] = tensor_scale_of(m, NVFP4);
             if (w == 0 && col0 + c < C) a.outer[(col0 + c) * (a.K / 128) + row0 / 128] = s_ref[cc];
         }
     }

@@ -133,10 +133,11 @@ fp4_status_t fp4_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int6
  *      MXFP4 (block 32): e = clamp(floor(log2 m) - 2, -127, 127) (m = 0:
  *        -127), byte e + 127, v = x * 2^-e;
  *      NVFP4 / UFP4 (block 16, Q = 6 / 7): s_t = A / (Q * 448) from the
- *        tensor amax A (1 if A = 0), s_b = E4M3_rne_satfinite((m / Q) / s_t),
+ *        tensor amax A (1 if that is 0: A = 0 or an underflowing quotient),
+ *        s_b = E4M3_rne_satfinite((m / Q) / s_t),
  *        v = x / (s_b * s_t); s_b = 0 gives signed zero codes;
  *      double block (NVFP4 only): s_o = m128 / 2688 per 128-element chunk of
- *        the line (1 if m128 = 0) replaces s_t;
+ *        the line (1 if that is 0) replaces s_t;
  *   4. round |v| onto the grid (clamped to the top level), sign from x:
  *      FP4_RTNE: nearest, ties to the even magnitude index;
  *      FP4_SR: up from the level below with probability (|v| - lo)/(hi - lo),

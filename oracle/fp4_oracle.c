@@ -32,7 +32,9 @@
  *   - MX scale exponent e = floor(log2 amax) - 2, clamped to [-127, 127];
  *     an all-zero block gets e = -127.
  *   - NV: s_t = amax/(6*448) (UFP4: amax/(7*448)), s_b = E4M3_RNE_sat((m/Q)/s_t),
- *     v = x / (s_b*s_t); a zero block scale gives signed zeros.
+ *     v = x / (s_b*s_t); a zero block scale gives signed zeros.  A tensor or
+ *     outer scale that comes out 0 (amax 0, or an amax below 2688 * 2^-149
+ *     whose quotient underflows) is replaced by 1, as for an all-zero block.
  *   - double block: s_o = amax128/2688 per 128-element chunk of a line,
  *     then the NV rule with s_t replaced by s_o.
  *   - rotation y = c_n * H_n * (d . x) on each aligned n-block of a line, H_n
@@ -297,7 +299,8 @@ static int floor_log2(float m)
 float orc_tensor_scale(float amax, int format)
 {
     float q448 = (format == ORC_UFP4) ? 7.0f * 448.0f : 6.0f * 448.0f;
-    return amax > 0.0f ? amax / q448 : 1.0f;
+    float s = amax / q448;
+    return s > 0.0f ? s : 1.0f;    /* amax 0, or so small the quotient underflows */
 }
 
 /* Quantize lines [l0, l1).  Outputs are indexed by line:
@@ -335,7 +338,8 @@ int orc_quantize_lines(const void* x, int in_dtype, int64_t R, int64_t C, int64_
                     float a = fabsf(buf[o * 128 + j]);
                     if (a > m128) m128 = a;
                 }
-                outer[lo * (K / 128) + o] = m128 > 0.0f ? m128 / 2688.0f : 1.0f;
+                float s_o = m128 / 2688.0f;
+                outer[lo * (K / 128) + o] = s_o > 0.0f ? s_o : 1.0f;   /* as for s_t */
             }
 
         for (int64_t b = 0; b < K / blk; ++b) {

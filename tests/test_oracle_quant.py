@@ -294,3 +294,18 @@ def test_rotation_changes_amax_and_matches_manual_blocks():
     manual = max(np.abs(oracle.rotate_block(x[r, 16 * b:16 * b + 16])).max()
                  for r in range(8) for b in range(4))
     assert amax == manual and amax < 100.0
+
+
+def test_underflowing_scales_fall_back_to_one():
+    """A tensor or outer scale amax/2688 that underflows to 0 is read as 1,
+    like the all-zero block: the codes are then signed zeros."""
+    tiny = np.float32(2.0 ** -149)
+    assert oracle.tensor_scale(float(tiny), oracle.NVFP4) == 1.0
+    assert oracle.tensor_scale(0.0, oracle.UFP4) == 1.0
+    x = np.full((2, 128), tiny, np.float32)
+    x[1] *= -1
+    q = oracle.quantize(x, oracle.NVFP4, double_block=True)
+    assert (q["outer"] == 1.0).all() and (q["scales"] == 0).all()
+    assert (q["codes"][0] == 0).all() and (q["codes"][1] == 0x88).all()
+    q = oracle.quantize(x, oracle.NVFP4)
+    assert q["tensor_scale"] == 1.0 and (q["scales"] == 0).all()
