@@ -133,13 +133,13 @@ def test_caller_given_amax(fp4):
     assert_quant_equal(g, o, what="given amax")
 
 
-def check_sampled(fp4, x_cpu, n_lines, seed, **kw):
+def check_sampled(fp4, x_cpu, n_lines, sample_seed, **kw):
     """Full-size GPU quantization, compared on sampled lines (the tensor amax
     is taken by the oracle over the whole tensor)."""
     axis = kw["axis"]
     L = x_cpu.shape[0] if axis == 1 else x_cpu.shape[1]
     g = gpu_quantize(fp4, x_cpu.cuda(), **kw)
-    lines = sample_lines(L, n_lines, seed)
+    lines = sample_lines(L, n_lines, sample_seed)
     o = oracle_quantize(x_cpu, lines=lines, **kw)
     assert_quant_equal(g, o, lines=lines, what="full-size " + str(kw))
     return g
