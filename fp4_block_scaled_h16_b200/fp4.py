@@ -32,7 +32,8 @@ FP4_IN_F32, FP4_IN_BF16 = 0, 1
 FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
 
 EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_quantize",
-           "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit")
+           "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit",
+           "fp4_quantize_noalloc")
 
 _P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_uint32, ctypes.c_size_t)
@@ -44,11 +45,12 @@ _lib.fp4_quantize_workspace_size.argtypes = [_I, _I, _I, ctypes.POINTER(_SZ)]
 _lib.fp4_amax.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _P, _P]
 _lib.fp4_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _I, _U64, _U32, _P,
                               _P, _P, _P, _P, _P, _SZ, _P]
+_lib.fp4_quantize_noalloc.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P]
 _lib.fp4_gemm.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P]
 _lib.fp4_last_error.argtypes = [_P]
 _lib.fp4_set_wait_limit.argtypes = [_U32]
 _lib.fp4_set_wait_limit.restype = None
-for _f in ("fp4_amax", "fp4_quantize", "fp4_gemm", "fp4_last_error", "fp4_quantize_workspace_size"):
+for _f in ("fp4_amax", "fp4_quantize", "fp4_quantize_noalloc", "fp4_gemm", "fp4_last_error", "fp4_quantize_workspace_size"):
     getattr(_lib, _f).restype = _I
 
 
@@ -111,6 +113,16 @@ def fp4_quantize(x, in_dtype, rows, cols, ld, fmt, rounding, rotation, axis, dou
                              int(double_block), seed, tensor_id, _ptr(tensor_amax), _ptr(codes),
                              _ptr(scales), _ptr(outer_scales), _ptr(tensor_scale), _ptr(workspace),
                              workspace_bytes, _stream(stream)), "fp4_quantize")
+
+
+def fp4_quantize_noalloc(x, in_dtype, rows, cols, ld, fmt, rounding, rotation, axis, seed, tensor_id,
+                         codes, scales, tensor_scale, stream=None) -> None:
+    """fp4_quantize (NVFP4 / UFP4, internal amax) without a workspace: the
+    scratch is the library's static device array.  For callers that cannot
+    allocate device memory; concurrent calls race on that array."""
+    _check(_lib.fp4_quantize_noalloc(_ptr(x), in_dtype, rows, cols, ld, fmt, rounding, rotation, axis, seed,
+                                     tensor_id, _ptr(codes), _ptr(scales), _ptr(tensor_scale), _stream(stream)),
+           "fp4_quantize_noalloc")
 
 
 def fp4_gemm(fmt, double_block, a_codes, a_scales, a_outer, a_tensor_scale, b_codes, b_scales,

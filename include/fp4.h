@@ -175,6 +175,37 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
                           void* stream);
 
 /*
+ * fp4_quantize_noalloc -- fp4_quantize for NVFP4 / UFP4 with the tensor scale
+ * taken from an internal amax, for callers that cannot allocate device
+ * memory: code running where cudaMalloc is unavailable or forbidden (a plug-in
+ * whose host framework owns every device allocation, a real-time loop that may
+ * not touch the allocator) and so cannot supply the 256-byte workspace
+ * fp4_quantize asks for.  The pages have no counterpart to this call; it only
+ * changes where the scratch lives.
+ *
+ * The scratch is a static device array of 256 bytes inside libfp4.so (one
+ * FP32 amax slot is used); every GPU that loads the library holds one copy
+ * until the process exits.  A request needing more scratch than that returns
+ * FP4_ERR_WORKSPACE (every NVFP4 / UFP4 shape needs exactly the 256 bytes).
+ * The caller still owns x, codes, scales and tensor_scale, with the layouts,
+ * shape rules and steps of fp4_quantize (double_block = 0, tensor_amax NULL).
+ * MXFP4 needs no scratch and returns FP4_ERR_UNSUPPORTED here: use
+ * fp4_quantize with no workspace.
+ *
+ * The first call on a device resolves the array's device address on that
+ * device (cudaGetSymbolAddress), so make it before any stream capture.  Every
+ * call shares the one array and leaves its amax there; each call clears the
+ * slot before accumulating into it.  Calls that overlap on the GPU (other
+ * streams, other threads, concurrent graph launches) race on the slot and
+ * must be serialized by the caller.  Allocates nothing; errors as
+ * fp4_quantize, checked before anything is launched.
+ */
+fp4_status_t fp4_quantize_noalloc(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols,
+                                  int64_t ld, fp4_format_t format, fp4_rounding_t rounding,
+                                  fp4_rotation_t rotation, int axis, uint64_t seed, uint32_t tensor_id,
+                                  uint8_t* codes, uint8_t* scales, float* tensor_scale, void* stream);
+
+/*
  * fp4_gemm -- block-scaled FP4 GEMM on tcgen05 tensor cores:
  *     C[i, j] = alpha_ij * sum_k qA[i, k] qB[j, k] sA[i, k/blk] sB[j, k/blk]
  * with A [M, K] and B [N, K] quantized tensors in the K-major view (lines
