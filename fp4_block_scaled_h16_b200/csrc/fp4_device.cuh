@@ -1,6 +1,6 @@
 // fp4_device.cuh -- device-side building blocks of the quantizer: Philox4x32-10,
-// the E2M1 / E4M3 conversions of sm_100a, the Sylvester butterfly and the
-// tiled scale-factor addressing.  Written for the CUDA path only.
+// the E2M1 / E4M3 conversions of sm_100a and the tiled scale-factor
+// addressing.  Written for the CUDA path only.
 #pragma once
 
 #include <cstdint>
@@ -74,35 +74,6 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// ---------------------------------------------------------------- exact division
-// q = RN(a / b) for a shared divisor b with precomputed y = RN(1/b):
-// q0 = RN(a*y), the remainder a - b*q0 is exact (FMA), then one correction.
-// Valid when b, 1/b and a/b stay in the normal range; the callers take
-// __fdiv_rn otherwise.
-__device__ __forceinline__ float div_by(float a, float b, float y) {
-    const float q0 = __fmul_rn(a, y);
-    const float r = __fmaf_rn(-b, q0, a);
-    return __fmaf_rn(r, y, q0);
-}
-
-// ---------------------------------------------------------------- butterfly
-// y = H_n x for n-element vectors held in registers, Sylvester order, stages
-// h = 1, 2, 4, ... ascending, every add / sub a single binary32 operation.
-template <int N>
-__device__ __forceinline__ void butterfly(float (&x)[N]) {
-#pragma unroll
-    for (int h = 1; h < N; h <<= 1) {
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-            if ((j & h) == 0) {
-                const float a = x[j], b = x[j + h];
-                x[j] = __fadd_rn(a, b);
-                x[j + h] = __fsub_rn(a, b);
-            }
-        }
-    }
-}
 
 // ---------------------------------------------------------------- tiled scales
 // byte offset of (line l, block b) in the tcgen05 scale-factor layout:

@@ -22,11 +22,15 @@ struct QuantArgs {
     PhiloxKeys keys;
     uint32_t tensor_id;
     uint32_t sign_mask;         // random-sign bits (0: deterministic Hadamard)
+    uint32_t div_m, div_l;      // multiply-shift division by the units per line (row kernel)
 };
 
-cudaError_t launch_quantize(const QuantArgs& a, bool bf16, int fmt, bool sr, int rot_n, bool db,
-                            int axis, cudaStream_t s);
-cudaError_t launch_amax(const QuantArgs& a, bool bf16, int rot_n, int axis, cudaStream_t s);
+cudaError_t launch_quantize(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, bool db, int axis,
+                            cudaStream_t s);
+cudaError_t launch_amax(QuantArgs a, bool bf16, int rot_n, int axis, cudaStream_t s);
+cudaError_t launch_quantize_cols(const QuantArgs& a, bool bf16, int fmt, bool sr, int rot_n, bool signs,
+                                 bool db, cudaStream_t s);
+cudaError_t launch_amax_cols(const QuantArgs& a, bool bf16, int rot_n, bool signs, cudaStream_t s);
 
 // GEMM
 struct GemmArgs {

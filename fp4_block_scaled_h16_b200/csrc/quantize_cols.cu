@@ -1,0 +1,214 @@
+// quantize_cols.cu -- the transposed-axis (axis = 0) quantizer: blocks run down
+// the columns of the row-major input and the output lines are its columns, as
+// the Dgrad / Wgrad operands need ("TetraJet-v2" 2.A: 1x16 groups re-aligned
+// for the transposed weight).  Same arithmetic as the row-axis kernel.
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "quant_common.cuh"
+
+namespace fp4 {
+
+// A CTA of 4 warps stages a 128-row x 64-column tile in shared memory; thread
+// (warp w, lane t) owns columns 2t, 2t+1 over rows 32w..32w+31, i.e. one
+// 32-element piece of two output lines, stored as 16 contiguous bytes each.
+constexpr int T0_ROWS = 128, T0_COLS = 64, T0_THREADS = 128;
+
+template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY>
+__global__ void __launch_bounds__(T0_THREADS)
+quant_cols_kernel(const QuantArgs a) {
+    __shared__ __align__(16) float tile[T0_ROWS][T0_COLS + 4];
+    __shared__ float chunk_max[4][T0_COLS];
+    const int64_t R = a.rows, C = a.cols;
+    const int64_t row0 = (int64_t)blockIdx.y * T0_ROWS, col0 = (int64_t)blockIdx.x * T0_COLS;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+
+    float s_t = 1.0f;
+    if (!AMAX_ONLY && FMT != MXFP4 && !DB) {
+        s_t = tensor_scale_of(*a.amax_in, FMT);
+        if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0 && a.tensor_scale_out) *a.tensor_scale_out = s_t;
+    }
+
+    // ---- stage the tile: 16-byte chunks, all loads issued first; zero outside [R, C)
+    constexpr int EPC = BF16 ? 8 : 4;                    // elements per 16-byte chunk
+    constexpr int CHUNKS = T0_ROWS * (T0_COLS / EPC);
+    constexpr int PER_THREAD = CHUNKS / T0_THREADS;
+    uint4 raw[PER_THREAD];
+#pragma unroll
+    for (int it = 0; it < PER_THREAD; ++it) {
+        const int q = tid + it * T0_THREADS;
+        const int r = q / (T0_COLS / EPC), c = (q % (T0_COLS / EPC)) * EPC;
+        const int64_t gr = row0 + r, gc = col0 + c;
+        if (gr < R && gc + EPC <= C) {
+            const uint4* p = BF16 ? reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.x) + gr * a.ld + gc)
+                                  : reinterpret_cast<const uint4*>(static_cast<const float*>(a.x) + gr * a.ld + gc);
+            raw[it] = __ldg(p);
+        } else {
+            uint32_t e[4] = {0u, 0u, 0u, 0u};
+            for (int k = 0; k < EPC; ++k) {
+                if (gr < R && gc + k < C) {
+                    const uint32_t bits = BF16 ? (uint32_t)__ldg(static_cast<const unsigned short*>(a.x) + gr * a.ld + gc + k)
+                                               : __float_as_uint(__ldg(static_cast<const float*>(a.x) + gr * a.ld + gc + k));
+                    if (BF16) e[k / 2] |= bits << (16 * (k & 1));
+                    else e[k] = bits;
+                }
+            }
+            raw[it] = make_uint4(e[0], e[1], e[2], e[3]);
+        }
+    }
+#pragma unroll
+    for (int it = 0; it < PER_THREAD; ++it) {
+        const int q = tid + it * T0_THREADS;
+        const int r = q / (T0_COLS / EPC), c = (q % (T0_COLS / EPC)) * EPC;
+        if (BF16) {
+            *reinterpret_cast<float4*>(&tile[r][c]) = make_float4(bf16_lo(raw[it].x), bf16_hi(raw[it].x),
+                                                                  bf16_lo(raw[it].y), bf16_hi(raw[it].y));
+            *reinterpret_cast<float4*>(&tile[r][c + 4]) = make_float4(bf16_lo(raw[it].z), bf16_hi(raw[it].z),
+                                                                      bf16_lo(raw[it].w), bf16_hi(raw[it].w));
+        } else {
+            *reinterpret_cast<float4*>(&tile[r][c]) = make_float4(__uint_as_float(raw[it].x), __uint_as_float(raw[it].y),
+                                                                  __uint_as_float(raw[it].z), __uint_as_float(raw[it].w));
+        }
+    }
+    __syncthreads();
+
+    const int64_t rbase = row0 + 32 * w;            // first row (= K index) of this piece
+    const int nvalid = (int)max((int64_t)0, min((int64_t)32, R - rbase));   // 0, 16 or 32
+    float v[2][32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float2 p = *reinterpret_cast<const float2*>(&tile[32 * w + k][2 * lane]);
+        v[0][k] = p.x;
+        v[1][k] = p.y;
+    }
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) rotate_unit<32, ROT, SIGNS>(v[cc], a.sign_mask);
+
+    if (AMAX_ONLY) {
+        // rows beyond R and columns beyond C are zero-filled and rotate to zero
+        const float m = absmax_n<32>(v[1], absmax_n<32>(v[0]));
+        const uint32_t bits = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+        if (lane == 0 && bits) atomicMax(a.amax_out, bits);
+        return;
+    }
+
+    float s_ref[2] = {s_t, s_t};
+    if (DB) {
+        // the 128-row chunk is this CTA's tile: reduce the 4 warps' maxima
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) chunk_max[w][2 * lane + cc] = absmax_n<32>(v[cc]);
+        __syncthreads();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * lane + cc;
+            const float m = fmaxf(fmaxf(chunk_max[0][c], chunk_max[1][c]), fmaxf(chunk_max[2][c], chunk_max[3][c]));
+            s_ref[cc] = tensor_scale_of(m, NVFP4);
+            if (w == 0 && col0 + c < C) a.outer[(col0 + c) * (a.K / 128) + row0 / 128] = s_ref[cc];
+        }
+    }
+    if (nvalid == 0) return;
+
+    uint32_t sbytes[2][2];
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        if (FMT == MXFP4) {
+            sbytes[cc][0] = mx_scale32(v[cc], absmax_n<32>(v[cc]));
+            sbytes[cc][1] = 1u;
+        } else {
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+                sbytes[cc][b] = nv_scale16<FMT>(v[cc] + 16 * b, absmax_n<16>(v[cc] + 16 * b), s_ref[cc]);
+        }
+    }
+    const int64_t line0 = col0 + 2 * lane;     // even; this thread's lines are line0, line0 + 1
+    uint32_t words[2][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t rnd[2][8];
+        if (SR) {
+            // element (r, line): i = r * C + line.  With C % 4 == 0 the two
+            // lines of a row share one Philox group (words line0 % 4 and +1).
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint64_t i = (uint64_t)(rbase + 8 * q + k) * (uint64_t)C + (uint64_t)line0;
+                const uint4 wds = sr_words(i >> 2, a.tensor_id, a.keys);
+                rnd[0][k] = word_of(wds, (int)(i & 3));
+                if ((C & 3) == 0) {
+                    rnd[1][k] = word_of(wds, (int)(i & 3) + 1);
+                } else {
+                    const uint64_t i1 = i + 1;
+                    rnd[1][k] = word_of(sr_words(i1 >> 2, a.tensor_id, a.keys), (int)(i1 & 3));
+                }
+            }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const bool z = (FMT != MXFP4) && sbytes[cc][q / 2] == 0u;
+            words[cc][q] = z ? sign_nibbles8(v[cc] + 8 * q) : encode8<FMT, SR>(v[cc] + 8 * q, rnd[cc]);
+        }
+    }
+    constexpr int BLK = (FMT == MXFP4) ? 32 : 16;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        const int64_t line = line0 + cc;
+        if (line < C) {
+            uint8_t* dst = a.codes + line * (a.K / 2) + rbase / 2;
+            if (nvalid == 32 && (a.K & 31) == 0) {
+                *reinterpret_cast<uint4*>(dst) = make_uint4(words[cc][0], words[cc][1], words[cc][2], words[cc][3]);
+            } else {
+                // line pitch K/2 is only 8-byte aligned when K % 32 == 16
+                reinterpret_cast<uint2*>(dst)[0] = make_uint2(words[cc][0], words[cc][1]);
+                if (nvalid == 32) reinterpret_cast<uint2*>(dst)[1] = make_uint2(words[cc][2], words[cc][3]);
+            }
+            a.scales[sf_offset(line, rbase / BLK, a.nb4)] = (uint8_t)sbytes[cc][0];
+            if (FMT != MXFP4 && nvalid == 32) a.scales[sf_offset(line, rbase / BLK + 1, a.nb4)] = (uint8_t)sbytes[cc][1];
+        }
+    }
+}
+
+// -------------------------------------------------------------------- dispatch
+
+namespace {
+
+template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY>
+cudaError_t launch_cols(const QuantArgs& a, cudaStream_t s) {
+    dim3 grid((unsigned)((a.cols + T0_COLS - 1) / T0_COLS), (unsigned)((a.rows + T0_ROWS - 1) / T0_ROWS));
+    quant_cols_kernel<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY><<<grid, T0_THREADS, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <bool BF16, int FMT, bool SR, bool DB, bool AMAX_ONLY>
+cudaError_t cols_by_rot(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s) {
+    if (rot_n == 0) return launch_cols<BF16, FMT, SR, 0, false, DB, AMAX_ONLY>(a, s);
+    if (rot_n == 16) return signs ? launch_cols<BF16, FMT, SR, 16, true, DB, AMAX_ONLY>(a, s)
+                                  : launch_cols<BF16, FMT, SR, 16, false, DB, AMAX_ONLY>(a, s);
+    return signs ? launch_cols<BF16, FMT, SR, 32, true, DB, AMAX_ONLY>(a, s)
+                 : launch_cols<BF16, FMT, SR, 32, false, DB, AMAX_ONLY>(a, s);
+}
+
+template <bool BF16>
+cudaError_t cols_by_fmt(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db, cudaStream_t s) {
+    if (fmt == MXFP4) return sr ? cols_by_rot<BF16, MXFP4, true, false, false>(a, rot_n, signs, s)
+                                : cols_by_rot<BF16, MXFP4, false, false, false>(a, rot_n, signs, s);
+    if (fmt == UFP4) return sr ? cols_by_rot<BF16, UFP4, true, false, false>(a, rot_n, signs, s)
+                               : cols_by_rot<BF16, UFP4, false, false, false>(a, rot_n, signs, s);
+    if (db) return sr ? cols_by_rot<BF16, NVFP4, true, true, false>(a, rot_n, signs, s)
+                      : cols_by_rot<BF16, NVFP4, false, true, false>(a, rot_n, signs, s);
+    return sr ? cols_by_rot<BF16, NVFP4, true, false, false>(a, rot_n, signs, s)
+              : cols_by_rot<BF16, NVFP4, false, false, false>(a, rot_n, signs, s);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_cols(const QuantArgs& a, bool bf16, int fmt, bool sr, int rot_n, bool signs,
+                                 bool db, cudaStream_t s) {
+    return bf16 ? cols_by_fmt<true>(a, fmt, sr, rot_n, signs, db, s)
+                : cols_by_fmt<false>(a, fmt, sr, rot_n, signs, db, s);
+}
+
+cudaError_t launch_amax_cols(const QuantArgs& a, bool bf16, int rot_n, bool signs, cudaStream_t s) {
+    return bf16 ? cols_by_rot<true, NVFP4, false, false, true>(a, rot_n, signs, s)
+                : cols_by_rot<false, NVFP4, false, false, true>(a, rot_n, signs, s);
+}
+
+}  // namespace fp4
