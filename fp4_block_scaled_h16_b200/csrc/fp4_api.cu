@@ -174,6 +174,7 @@ fp4_status_t fp4_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int6
     a.K = axis ? cols : rows;
     a.amax_out = reinterpret_cast<unsigned int*>(amax_out);
     a.sign_mask = sign_mask_of(rotation, seed);
+    a.err = device_error_word();
     if (launch_amax(a, in_dtype == FP4_IN_BF16, rot_size(rotation), axis, s) != cudaSuccess) return FP4_ERR_CUDA;
     return FP4_OK;
 }
@@ -228,6 +229,7 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
     a.keys = make_keys(seed);
     a.tensor_id = tensor_id;
     a.sign_mask = sign_mask_of(rotation, seed);
+    a.err = device_error_word();
     const int rn = rot_size(rotation);
     const bool bf16 = in_dtype == FP4_IN_BF16;
     if (internal_amax) {

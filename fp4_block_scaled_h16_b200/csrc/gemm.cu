@@ -125,7 +125,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (sm100::elect_one()) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t fills[STAGES] = {};
+            uint32_t fills = 0;           // fill i went to stage i % STAGES, phase i / STAGES
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN;
@@ -148,13 +148,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                         sm100::bulk_load(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES + rb * G::ATOMS * 512,
                                          sfb, G::ATOMS * 512, &full[stage]);
                     }
-                    fills[stage]++;
+                    ++fills;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            // drain: every fill issued must land before the CTA may exit
+            // drain: every fill issued must land before the CTA may exit; the
+            // last fill of stage s had phase (fills - 1 - s) / STAGES
+#pragma unroll
             for (int s = 0; s < STAGES; ++s)
-                if (fills[s]) sm100::mbar_wait(&full[s], (fills[s] - 1) & 1u, DRAIN_LIMIT, nullptr);
+                if (fills > (uint32_t)s)
+                    sm100::mbar_wait(&full[s], ((fills - 1u - s) / STAGES) & 1u, DRAIN_LIMIT, nullptr);
         }
         __syncwarp();
     } else if (warp == 1) {

@@ -22,7 +22,8 @@ struct QuantArgs {
     PhiloxKeys keys;
     uint32_t tensor_id;
     uint32_t sign_mask;         // random-sign bits (0: deterministic Hadamard)
-    uint32_t div_m, div_l;      // multiply-shift division by the units per line (row kernel)
+    uint32_t div_m, div_l;      // multiply-shift division by the units per line
+    unsigned int* err;          // device error word (a bounded wait that ran out)
 };
 
 cudaError_t launch_quantize(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, bool db, int axis,

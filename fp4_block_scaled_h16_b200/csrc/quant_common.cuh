@@ -110,6 +110,49 @@ __device__ __forceinline__ void rotate_block(float* v, uint32_t sign_mask) {
     }
 }
 
+// max |y| of a rotated block without materialising y: max_j |RN(c*y_j)| =
+// RN(c * max_j |y_j|) (c > 0 and rounding are monotone), and the last stage's
+// pair (a + b, a - b) has max(|RN(a+b)|, |RN(a-b)|) = RN(|a| + |b|).
+template <int N, bool SIGNS>
+__device__ __forceinline__ float rotated_absmax(const float* v, uint32_t sign_mask, float m) {
+    constexpr int H = N / 2;
+    float2 p[H];
+#pragma unroll
+    for (int i = 0; i < H; ++i) {
+        float a = v[i], b = v[i + H];
+        if (SIGNS) {
+            a = __uint_as_float(__float_as_uint(a) ^ (((sign_mask >> i) & 1u) << 31));
+            b = __uint_as_float(__float_as_uint(b) ^ (((sign_mask >> (i + H)) & 1u) << 31));
+        }
+        p[i] = make_float2(a, b);
+    }
+#pragma unroll
+    for (int h = 1; h < H; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+            if ((i & h) == 0) {
+                const float2 a = p[i], b = p[i + h];
+                p[i] = add2(a, b);
+                p[i + h] = sub2(a, b);
+            }
+        }
+    }
+    float t = 0.0f;
+#pragma unroll
+    for (int i = 0; i + 1 < H; i += 2)
+        t = amax3(t, __fadd_rn(fabsf(p[i].x), fabsf(p[i].y)), __fadd_rn(fabsf(p[i + 1].x), fabsf(p[i + 1].y)));
+    const float c = (N == 16) ? 0.25f : __uint_as_float(0x3E3504F3u);
+    return fmaxf(m, __fmul_rn(t, c));
+}
+
+template <int U, int ROT, bool SIGNS>
+__device__ __forceinline__ float unit_rotated_absmax(const float* v, uint32_t sign_mask, float m) {
+    if (ROT == 0) return absmax_n<U>(v, m);
+#pragma unroll
+    for (int b = 0; b < U / (ROT ? ROT : 16); ++b) m = rotated_absmax<(ROT ? ROT : 16), SIGNS>(v + b * ROT, sign_mask, m);
+    return m;
+}
+
 template <int U, int ROT, bool SIGNS>
 __device__ __forceinline__ void rotate_unit(float* v, uint32_t sign_mask) {
     if (ROT) {
@@ -119,17 +162,29 @@ __device__ __forceinline__ void rotate_unit(float* v, uint32_t sign_mask) {
 }
 
 // ------------------------------------------------------------------ scales
+// Pair layout of a unit: packed operations act on (v[j], v[j + PS]), with
+// PS = 8 under a 16-rotation (the rotation's own pairs) and U/2 otherwise.
+template <int U, int ROT>
+struct PairLayout {
+    static constexpr int PS = (ROT == 16 || U == 16) ? 8 : U / 2;
+    static constexpr int N = U / 2;                       // pairs per unit
+    static __device__ __forceinline__ int lo(int p) { return PS == 8 ? (p & 7) + ((p >> 3) << 4) : p; }
+};
+
 // MX: e = clamp(floor(log2 m) - 2, -127, 127); v <- v * 2^-e (exact); returns e + 127
+template <int ROT>
 __device__ __forceinline__ uint32_t mx_scale32(float* v, float m) {
+    using PL = PairLayout<32, ROT>;
     int e = (m > 0.0f) ? ilogbf(m) - 2 : -127;
     e = max(-127, min(127, e));
     const float inv = (e <= 126) ? __uint_as_float((uint32_t)(127 - e) << 23) : __uint_as_float(0x00400000u);
     const float2 ii = make_float2(inv, inv);
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-        const float2 r = mul2(make_float2(v[j], v[j + 1]), ii);
+    for (int p = 0; p < PL::N; ++p) {
+        const int j = PL::lo(p);
+        const float2 r = mul2(make_float2(v[j], v[j + PL::PS]), ii);
         v[j] = r.x;
-        v[j + 1] = r.y;
+        v[j + PL::PS] = r.y;
     }
     return (uint32_t)(e + 127);
 }
@@ -141,33 +196,82 @@ __device__ __forceinline__ float tensor_scale_of(float amax, int fmt) {
     return s > 0.0f ? s : 1.0f;
 }
 
-// NV / UFP4 16-block: s_b = E4M3((m / Q) / s_ref); v <- v / (s_b * s_ref).
-// Returns the scale byte (0: the block is all signed zeros, v untouched).
+// RN(a / d) from y = RN(1/d) by one correction step: q0 = a*y, r = a - d*q0
+// (exact), q = q0 + r*y.  Exact while a, d, 1/d and the quotient are normal;
+// for d = 6 and d = 7 an exhaustive check over every normal a >= 2^-122
+// agrees with IEEE division.
+__device__ __forceinline__ float div_rcp(float a, float d, float y) {
+    const float q0 = __fmul_rn(a, y);
+    return __fmaf_rn(__fmaf_rn(-d, q0, a), y, q0);
+}
+
+// per-tensor (or per-chunk) reference scale with its reciprocal, for the block scale
+struct ScaleRef {
+    float s, y;        // s_ref and RN(1/s_ref)
+    bool fast;         // s_ref in [2^-100, 2^100]: the correction step is exact
+};
+__device__ __forceinline__ ScaleRef make_ref(float s) {
+    ScaleRef r;
+    r.s = s;
+    r.fast = (s >= 0x1p-100f) && (s <= 0x1p100f);
+    r.y = r.fast ? __frcp_rn(s) : 0.0f;
+    return r;
+}
+
+// s_b = E4M3_rne_satfinite((m / Q) / s_ref), both divisions correctly rounded
 template <int FMT>
-__device__ __forceinline__ uint32_t nv_scale16(float* v, float m, float s_ref) {
+__device__ __forceinline__ uint32_t block_scale_code(float m, const ScaleRef& ref) {
     constexpr float Q = (FMT == UFP4) ? 7.0f : 6.0f;
-    const float sb = __fdiv_rn(__fdiv_rn(m, Q), s_ref);
-    const uint32_t E = cvt_e4m3(sb);
-    if (E == 0u) return 0u;
+    constexpr float YQ = (FMT == UFP4) ? 0x1.24924ap-3f : 0x1.555556p-3f;   // RN(1/7), RN(1/6)
+    const float n = (m >= 0x1p-122f) ? div_rcp(m, Q, YQ) : __fdiv_rn(m, Q);
+    float sb;
+    if (ref.fast && n >= 0x1p-100f && __fmul_rn(n, ref.y) < 0x1p100f) sb = div_rcp(n, ref.s, ref.y);
+    else sb = __fdiv_rn(n, ref.s);
+    return cvt_e4m3(sb);
+}
+
+// S = RN(E * s_ref) and y = RN(1/S) for block scale code E; y = 0 marks a
+// block that takes the slow path: IEEE division when S or 1/S is outside the
+// normal range, and, for E = 0 (S = 0), x * 0, the signed zeros of the codes.
+__device__ __forceinline__ float2 scale_pair(uint32_t E, float s_ref) {
+    if (E == 0u) return make_float2(0.0f, 0.0f);
     const float S = __fmul_rn(e4m3_to_f32(E), s_ref);
-    if (S >= 0x1p-125f && S <= 0x1p125f) {
-        // q0 = x*y, r = x - S*q0 (exact), q = q0 + r*y: RN(x / S) for this range
-        const float y = __frcp_rn(S);
-        const float2 yy = make_float2(y, y), ns = make_float2(-S, -S);
+    const bool fast = S >= 0x1p-125f && S <= 0x1p125f;
+    return make_float2(S, fast ? __frcp_rn(S) : 0.0f);
+}
+
+// per-CTA table of scale_pair(E, s_t) for every E4M3 code of a tensor scale
+struct ScaleTable {
+    float2 e[128];
+    __device__ __forceinline__ void build(float s_t, int tid, int nthreads) {
+        for (int c = tid; c < 128; c += nthreads) e[c] = scale_pair((uint32_t)c, s_t);
+    }
+};
+
+// v <- v / S per element, S and y per 16-block (SY[b] = (S_b, y_b)), on the
+// unit's pair layout: q0 = x*y, r = x - S*q0 (exact), q = q0 + r*y = RN(x/S)
+// while S and 1/S are normal; IEEE division otherwise; S = y = 0 -> +-0.
+template <int U, int ROT>
+__device__ __forceinline__ void nv_divide(float* v, const float2* SY) {
+    using PL = PairLayout<U, ROT>;
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-            const float2 x = make_float2(v[j], v[j + 1]);
+    for (int p = 0; p < PL::N; ++p) {
+        const int j = PL::lo(p), k = j + PL::PS;
+        const float2 a = SY[j / 16], b = SY[k / 16];
+        const bool slow = (a.y == 0.0f) || (b.y == 0.0f);
+        if (!slow) {
+            const float2 x = make_float2(v[j], v[k]);
+            const float2 yy = make_float2(a.y, b.y);
             const float2 q0 = mul2(x, yy);
-            const float2 r = __ffma2_rn(ns, q0, x);
+            const float2 r = __ffma2_rn(make_float2(-a.x, -b.x), q0, x);
             const float2 q = __ffma2_rn(r, yy, q0);
             v[j] = q.x;
-            v[j + 1] = q.y;
+            v[k] = q.y;
+        } else {
+            v[j] = a.x != 0.0f ? __fdiv_rn(v[j], a.x) : __fmul_rn(v[j], 0.0f);
+            v[k] = b.x != 0.0f ? __fdiv_rn(v[k], b.x) : __fmul_rn(v[k], 0.0f);
         }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __fdiv_rn(v[j], S);
     }
-    return E;
 }
 
 // ------------------------------------------------------------------ encoders
@@ -211,11 +315,16 @@ __device__ __forceinline__ uint32_t encode8(const float* v, const uint32_t* rnd)
     if (FMT != UFP4 && !SR) {
         // hardware RNE onto E2M1, saturating at +-6; a value rounding to zero
         // keeps its sign (code 8), as the method's codes require
-        const uint32_t b0 = cvt_e2m1x2(v[0], v[1]);
-        const uint32_t b1 = cvt_e2m1x2(v[2], v[3]);
-        const uint32_t b2 = cvt_e2m1x2(v[4], v[5]);
-        const uint32_t b3 = cvt_e2m1x2(v[6], v[7]);
-        return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        uint32_t w;
+        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+            "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+            : "=r"(w)
+            : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+        return w;
     }
     uint32_t w = 0;
 #pragma unroll

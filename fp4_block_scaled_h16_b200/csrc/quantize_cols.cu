@@ -23,10 +23,12 @@ quant_cols_kernel(const QuantArgs a) {
     const int64_t row0 = (int64_t)blockIdx.y * T0_ROWS, col0 = (int64_t)blockIdx.x * T0_COLS;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
 
-    float s_t = 1.0f;
+    __shared__ ScaleTable table;                        // (S, 1/S) per E4M3 code under s_t
+    ScaleRef ref_t = make_ref(1.0f);
     if (!AMAX_ONLY && FMT != MXFP4 && !DB) {
-        s_t = tensor_scale_of(*a.amax_in, FMT);
-        if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0 && a.tensor_scale_out) *a.tensor_scale_out = s_t;
+        ref_t = make_ref(tensor_scale_of(*a.amax_in, FMT));
+        if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0 && a.tensor_scale_out) *a.tensor_scale_out = ref_t.s;
+        table.build(ref_t.s, tid, T0_THREADS);
     }
 
     // ---- stage the tile: 16-byte chunks, all loads issued first; zero outside [R, C)
@@ -92,7 +94,7 @@ quant_cols_kernel(const QuantArgs a) {
         return;
     }
 
-    float s_ref[2] = {s_t, s_t};
+    ScaleRef s_ref[2] = {ref_t, ref_t};
     if (DB) {
         // the 128-row chunk is this CTA's tile: reduce the 4 warps' maxima
 #pragma unroll
@@ -102,8 +104,8 @@ quant_cols_kernel(const QuantArgs a) {
         for (int cc = 0; cc < 2; ++cc) {
             const int c = 2 * lane + cc;
             const float m = fmaxf(fmaxf(chunk_max[0][c], chunk_max[1][c]), fmaxf(chunk_max[2][c], chunk_max[3][c]));
-            s_ref[cc] = tensor_scale_of(m, NVFP4);
-            if (w == 0 && col0 + c < C) a.outer[(col0 + c) * (a.K / 128) + row0 / 128] = s_ref[cc];
+            s_ref[cc] = make_ref(tensor_scale_of(m, NVFP4));
+            if (w == 0 && col0 + c < C) a.outer[(col0 + c) * (a.K / 128) + row0 / 128] = s_ref[cc].s;
         }
     }
     if (nvalid == 0) return;
@@ -112,12 +114,16 @@ quant_cols_kernel(const QuantArgs a) {
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
         if (FMT == MXFP4) {
-            sbytes[cc][0] = mx_scale32(v[cc], absmax_n<32>(v[cc]));
+            sbytes[cc][0] = mx_scale32<ROT>(v[cc], absmax_n<32>(v[cc]));
             sbytes[cc][1] = 1u;
         } else {
+            float2 SY[2];
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
-                sbytes[cc][b] = nv_scale16<FMT>(v[cc] + 16 * b, absmax_n<16>(v[cc] + 16 * b), s_ref[cc]);
+            for (int b = 0; b < 2; ++b) {
+                sbytes[cc][b] = block_scale_code<FMT>(absmax_n<16>(v[cc] + 16 * b), s_ref[cc]);
+                SY[b] = DB ? scale_pair(sbytes[cc][b], s_ref[cc].s) : table.e[sbytes[cc][b]];
+            }
+            nv_divide<32, ROT>(v[cc], SY);
         }
     }
     const int64_t line0 = col0 + 2 * lane;     // even; this thread's lines are line0, line0 + 1
@@ -142,10 +148,7 @@ quant_cols_kernel(const QuantArgs a) {
             }
         }
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const bool z = (FMT != MXFP4) && sbytes[cc][q / 2] == 0u;
-            words[cc][q] = z ? sign_nibbles8(v[cc] + 8 * q) : encode8<FMT, SR>(v[cc] + 8 * q, rnd[cc]);
-        }
+        for (int cc = 0; cc < 2; ++cc) words[cc][q] = encode8<FMT, SR>(v[cc] + 8 * q, rnd[cc]);
     }
     constexpr int BLK = (FMT == MXFP4) ? 32 : 16;
 #pragma unroll
