@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "fp4_device.cuh"
@@ -52,6 +53,9 @@ struct GemmArgs {
     uint32_t wait_limit;
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+cudaError_t launch_gemm_db(const GemmArgs& g, cudaStream_t s);
+// 2-D TMA map over packed codes [rows, K/2] bytes: box 128 bytes x box_rows, 128-byte swizzle
+bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K, int box_rows);
 
 // device state
 int num_sms();

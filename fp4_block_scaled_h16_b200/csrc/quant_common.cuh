@@ -147,9 +147,12 @@ __device__ __forceinline__ float rotated_absmax(const float* v, uint32_t sign_ma
 
 template <int U, int ROT, bool SIGNS>
 __device__ __forceinline__ float unit_rotated_absmax(const float* v, uint32_t sign_mask, float m) {
-    if (ROT == 0) return absmax_n<U>(v, m);
+    if (ROT == 0) {
+        m = absmax_n<U>(v, m);
+    } else {
 #pragma unroll
-    for (int b = 0; b < U / (ROT ? ROT : 16); ++b) m = rotated_absmax<(ROT ? ROT : 16), SIGNS>(v + b * ROT, sign_mask, m);
+        for (int b = 0; b < U / (ROT ? ROT : 16); ++b) m = rotated_absmax<(ROT ? ROT : 16), SIGNS>(v + b * ROT, sign_mask, m);
+    }
     return m;
 }
 

@@ -125,9 +125,38 @@ def test_full_mxfp4_wgrad_down(fp4):
     sampled_gemm_check(fp4, qa, qb, d["dY"], d["H"], ka, kb, False, 96, 1)
 
 
-def test_double_block_gemm_not_yet(fp4):
-    a = rand(128, 512, 1)
+@pytest.mark.parametrize("out_bf16", [False, True])
+@pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 512), (128, 256, 2048), (384, 128, 8192)])
+def test_double_block_gemm_on_oracle_operands(fp4, out_bf16, shape):
+    """C = sum over 128-K chunks of s_oA * s_oB * (block-scaled partial)."""
+    M, N, K = shape
+    a, b = rand(M, K, M + K), rand(N, K, 7 * N + K, 0.1)
+    # chunk magnitudes that vary along K, so every chunk's outer scale matters
+    a = a * torch.from_numpy(np.repeat(np.exp2(np.random.default_rng(1).integers(-6, 6, K // 128)), 128)).float()
+    qa = oracle_quantize(a, fmt=NV, double_block=True, rounding=1, seed=3, tensor_id=1)
+    qb = oracle_quantize(b, fmt=NV, double_block=True, rounding=1, seed=3, tensor_id=2)
+    C64, bound = oracle.gemm(qa, qb)
+    C = fp4.gemm(upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb),
+                 fp4.FP4_OUT_BF16 if out_bf16 else fp4.FP4_OUT_F32)
+    torch.cuda.synchronize()
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    assert_within_gemm_bound(C.float().cpu().numpy(), C64, bound, out_bf16, what="db %s" % (shape,))
+
+
+def test_full_nvfp4_dgrad_double_block(fp4):
+    """dH = dY Wd: dY 8192x4096 (axis 1), Wd 4096x14336 quantized along its
+    transposed axis (axis 0), double block, SR; bf16 out 8192x14336."""
+    d = workloads.nvfp4_dgrad_down()
+    ka = dict(fmt=NV, rounding=1, rotation=0, axis=1, double_block=True, seed=0, tensor_id=1)
+    kb = dict(fmt=NV, rounding=1, rotation=0, axis=0, double_block=True, seed=0, tensor_id=2)
+    qa = fp4.quantize(d["dY"].cuda(), **ka)
+    qb = fp4.quantize(d["Wd"].cuda(), **kb)
+    sampled_gemm_check(fp4, qa, qb, d["dY"], d["Wd"], ka, kb, True, 96, 2)
+
+
+def test_double_block_gemm_rejects_long_k(fp4):
+    a = rand(128, 8448, 1)
     qa = fp4.quantize(a.cuda(), fmt=NV, double_block=True)
     with pytest.raises(fp4.Fp4Error) as e:
         fp4.gemm(qa, qa)
-    assert e.value.status == fp4.FP4_ERR_UNSUPPORTED
+    assert e.value.status == fp4.FP4_ERR_UNSUPPORTED_SHAPE
