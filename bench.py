@@ -251,6 +251,117 @@ def run_gpu(args, rank, world, device):
     return line
 
 
+# ------------------------------------------------------------------------ every config
+
+def _median_ms(fn, flush, reps):
+    """Median CUDA-event time of fn() over reps runs, L2 flushed before each."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
+def _qbytes(x, fmt, db):
+    """Algorithmic bytes of one quantize call: read once, codes + scales (+ outer) written."""
+    n = x.numel()
+    blk = 32 if fmt == 0 else 16
+    return n * x.element_size() + n / 2 + n / blk + (n / 128 * 4 if db else 0)
+
+
+def measure_configs(fp4, device, peaks, reps=10):
+    """Per-kernel timings of every workload: quantize GB/s and GEMM TFLOP/s with
+    their fractions of the measured HBM and derived FP4 peaks."""
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    fp4_peak = peaks["bf16"] * 4.0
+    out = {}
+
+    def quant_entry(x, **kw):
+        fmt, db = kw["fmt"], kw.get("double_block", False)
+        axis = kw.get("axis", 1)
+        R, C = x.shape
+        q = fp4.alloc_qtensor(R if axis else C, C if axis else R, fmt, db, device)
+        ws = torch.empty(256, dtype=torch.uint8, device=device)
+        ms = _median_ms(lambda: fp4.quantize(x, out=q, workspace=ws, **kw), flush, reps)
+        gb = _qbytes(x, fmt, db) + (x.numel() * x.element_size() if (fmt != 0 and not db) else 0)
+        return q, {"ms": ms, "gbs": gb / (ms * 1e6), "frac_hbm": gb / (ms * 1e6) / peaks["hbm"],
+                   "bytes": "2 reads (amax pass + quantize)" if (fmt != 0 and not db) else "1 read"}
+
+    def gemm_entry(qa, qb, out_dtype):
+        M, N, K = qa["lines"], qb["lines"], qa["K"]
+        C = torch.empty((M, N), dtype=torch.bfloat16 if out_dtype else torch.float32, device=device)
+        ms = _median_ms(lambda: fp4.gemm(qa, qb, out_dtype, out=C), flush, reps)
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        return {"ms": ms, "tflops": tf, "frac_fp4": tf / fp4_peak, "shape": [M, N, K]}
+
+    NV, MX, UF = fp4.FP4_NVFP4, fp4.FP4_MXFP4, fp4.FP4_UFP4
+    BF, F32 = fp4.FP4_OUT_BF16, fp4.FP4_OUT_F32
+
+    d = workloads.tiny_mxfp4()
+    A, B = d["A"].to(device), d["B"].to(device)
+    qa, ea = quant_entry(A, fmt=MX, axis=1)
+    qb, eb = quant_entry(B, fmt=MX, axis=0)
+    out["tiny_mxfp4_256x256x512"] = {"quantize_A": ea, "quantize_B": eb, "gemm": gemm_entry(qa, qb, F32),
+                                     "note": "launch-bound; outside the roofline targets"}
+
+    d = workloads.mxfp4_wgrad_down()
+    dY, H = d["dY"].to(device), d["H"].to(device)
+    kw = dict(fmt=MX, rounding=fp4.FP4_SR, rotation=fp4.FP4_ROT_RH32, axis=0, seed=0)
+    qa, ea = quant_entry(dY, tensor_id=1, **kw)
+    qb, eb = quant_entry(H, tensor_id=2, **kw)
+    out["mxfp4_wgrad_down_4096x14336x8192"] = {"quantize_dY": ea, "quantize_H": eb, "gemm": gemm_entry(qa, qb, F32)}
+    del dY, H, qa, qb
+
+    d = workloads.nvfp4_dgrad_down()
+    dY, Wd = d["dY"].to(device), d["Wd"].to(device)
+    kw = dict(fmt=NV, rounding=fp4.FP4_SR, double_block=True, seed=0)
+    qa, ea = quant_entry(dY, axis=1, tensor_id=1, **kw)
+    qb, eb = quant_entry(Wd, axis=0, tensor_id=2, **kw)
+    out["nvfp4_dgrad_down_db_8192x14336x4096"] = {"quantize_dY": ea, "quantize_Wd": eb, "gemm": gemm_entry(qa, qb, BF)}
+    del dY, Wd, qa, qb
+
+    # the decoder layer: Fprop, Dgrad, Wgrad of each linear in NVFP4 with H16
+    # (SR on the Wgrad operands), then the UFP4 quantizer on the same operands
+    layer = {"quantize_nvfp4_ms": 0.0, "quantize_ufp4_ms": 0.0, "quantize_bytes": 0.0, "gemm_ms": 0.0,
+             "gemm_flop": 0.0, "linears": {}}
+    for name, _, _, _ in workloads.LAYER_LINEARS:
+        d = workloads.layer_linear(name)
+        X, W, dY = d["X"].to(device), d["W"].to(device), d["dY"].to(device)
+        H16, SR, RT = fp4.FP4_ROT_H16, fp4.FP4_SR, fp4.FP4_RTNE
+        ops = {"X_ax1": (X, 1, RT), "W_ax1": (W, 1, RT), "dY_ax1": (dY, 1, RT), "W_ax0": (W, 0, RT),
+               "dY_ax0": (dY, 0, SR), "X_ax0": (X, 0, SR)}
+        lin = {}
+        qs = {}
+        for role, (t, axis, rnd) in ops.items():
+            qs[role], e = quant_entry(t, fmt=NV, rounding=rnd, rotation=H16, axis=axis, seed=0, tensor_id=len(qs))
+            _, u = quant_entry(t, fmt=UF, rounding=rnd, rotation=H16, axis=axis, seed=0, tensor_id=len(qs))
+            lin["nv_" + role], lin["uf_" + role] = e, u
+            layer["quantize_nvfp4_ms"] += e["ms"]
+            layer["quantize_ufp4_ms"] += u["ms"]
+            layer["quantize_bytes"] += e["gbs"] * e["ms"] * 1e6
+        for gname, (a_, b_, od) in {"fprop": ("X_ax1", "W_ax1", BF), "dgrad": ("dY_ax1", "W_ax0", BF),
+                                    "wgrad": ("dY_ax0", "X_ax0", F32)}.items():
+            g = gemm_entry(qs[a_], qs[b_], od)
+            lin[gname] = g
+            layer["gemm_ms"] += g["ms"]
+            layer["gemm_flop"] += 2.0 * g["shape"][0] * g["shape"][1] * g["shape"][2]
+        layer["linears"][name] = lin
+        del X, W, dY, qs
+        torch.cuda.empty_cache()
+    layer["gemm_tflops"] = layer["gemm_flop"] / (layer["gemm_ms"] * 1e-3) / 1e12
+    layer["gemm_frac_fp4"] = layer["gemm_tflops"] / fp4_peak
+    layer["quantize_nvfp4_gbs"] = layer["quantize_bytes"] / (layer["quantize_nvfp4_ms"] * 1e6)
+    layer["quantize_nvfp4_frac_hbm"] = layer["quantize_nvfp4_gbs"] / peaks["hbm"]
+    out["llama8b_layer_linears_t8192"] = layer
+    return out
+
+
 # ------------------------------------------------------------------------ oracle arm
 
 def oracle_slab_time(d, rows):
@@ -326,6 +437,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["fp4", "reference"], default="fp4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel table")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -346,6 +458,9 @@ def main():
                                              device_id=device)
     line = run_gpu(args, rank, world, device)
     if rank == 0:
+        if world == 1 and not args.no_configs:
+            from fp4_block_scaled_h16_b200 import fp4 as _fp4
+            line["configs"] = measure_configs(_fp4, device, measured_peaks())
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(workloads.nvfp4_fprop_qkv(seed=0))
         print(json.dumps(line), flush=True)

@@ -13,8 +13,11 @@
 //   warp 1   allocates TMEM and issues, from one thread, the smem->TMEM
 //            scale-factor copies and four 128 x BN x 64 block-scaled MMAs per
 //            stage into an FP32 accumulator in TMEM;
-//   warps 2-5 epilogue: TMEM -> registers (tcgen05.ld), times alpha, convert,
-//            store to global.
+//   warps 2-9 epilogue: two warps per TMEM lane quarter, each owning half of
+//            the tile's columns; all of a warp's TMEM loads are issued back to
+//            back, the accumulator is released to the MMA warp, and only then
+//            are the values scaled by alpha, converted and stored, so the
+//            stores overlap the next tile's mainloop.
 // Every mbarrier wait is bounded; a wait that runs out sets the device error
 // word to FP4_ERR_TIMEOUT, the CTA stops, lets every copy and MMA it issued
 // land, frees its TMEM and exits.
@@ -35,7 +38,8 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 256;                 // K elements per stage (128 bytes of codes per row)
 constexpr int STAGES = 4;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t DRAIN_LIMIT = 1u << 22;
 constexpr unsigned int ERR_TIMEOUT = 7u;   // FP4_ERR_TIMEOUT
@@ -101,7 +105,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             sm100::mbar_init(&empty[s], 1);
         }
         sm100::mbar_init(acc_full, 1);
-        sm100::mbar_init(acc_empty, 4);
+        sm100::mbar_init(acc_empty, EPI_WARPS);
         sm100::mbar_init(drain, 1);
         *abort_flag = 0;
         sm100::fence_barrier_init();
@@ -223,12 +227,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
+        constexpr int COLS = BN / 2;            // columns per epilogue warp
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;       // which half of the tile's columns
         float alpha = 1.0f;
         if (FMT == NVFP4) alpha = __fmul_rn(*p.a_ts, *p.b_ts);
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN;
+            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN + half * COLS;
             // one lane polls, the warp follows its verdict (the TMEM loads below
             // are warp-collective)
             int got = 0;
@@ -238,37 +244,40 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             }
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
             sm100::tc_fence_after();
-            const int row = m0 + 32 * q + lane;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 32 * c, r);
-                sm100::tmem_ld_wait();
-                if (OUT_BF16) {
-                    uint32_t pk[16];
+            uint32_t r[COLS];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * e]), alpha),
-                                                                       __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha));
-                        pk[e] = *reinterpret_cast<const uint32_t*>(&h);
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + n0 + 32 * c);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)row * p.ldc + n0 + 32 * c);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        dst[v] = make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha),
-                                             __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
-                                             __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
-                                             __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
-                }
+            for (int c = 0; c < COLS / 32; ++c) {
+                uint32_t (&rr)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[32 * c]);
+                sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + half * COLS + 32 * c, rr);
             }
+            sm100::tmem_ld_wait();
             sm100::tc_fence_before();
             __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(acc_empty);
+            if (lane == 0) sm100::mbar_arrive(acc_empty);          // the MMA may overwrite it now
             acc_phase ^= 1u;
+            const int row = m0 + 32 * q + lane;
+            if (OUT_BF16) {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + n0);
+#pragma unroll
+                for (int v = 0; v < COLS / 8; ++v) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[8 * v + 2 * e]), alpha),
+                                                                       __fmul_rn(__uint_as_float(r[8 * v + 2 * e + 1]), alpha));
+                        pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            } else {
+                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)row * p.ldc + n0);
+#pragma unroll
+                for (int v = 0; v < COLS / 4; ++v)
+                    dst[v] = make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha),
+                                         __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
+                                         __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
+                                         __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+            }
         }
     }
 
