@@ -30,7 +30,9 @@ namespace {
 
 constexpr int BM = 128, BN = 128, BK = 256;
 constexpr int STAGES = 4;
-constexpr int NUM_THREADS = 224;         // producer, MMA, 4 epilogue warps, outer-scale warp
+constexpr int EPI_WARPS = 8;              // two per TMEM lane quarter, half of the columns each
+constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS + 1);   // producer, MMA, epilogue, outer-scale warp
+constexpr int STAGER_WARP = 2 + EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t DRAIN_LIMIT = 1u << 22;
 constexpr unsigned int ERR_TIMEOUT = 7u;
@@ -89,9 +91,9 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         for (int b = 0; b < 2; ++b) {
             sm100::mbar_init(&pfull[b], 1);
-            sm100::mbar_init(&pempty[b], 4);
+            sm100::mbar_init(&pempty[b], EPI_WARPS);
             sm100::mbar_init(&ofull[b], 32);
-            sm100::mbar_init(&oempty[b], 4);
+            sm100::mbar_init(&oempty[b], EPI_WARPS);
         }
         sm100::mbar_init(drain, 1);
         *abort_flag = 0;
@@ -199,7 +201,7 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
         }
         __syncwarp();
-    } else if (warp == 6) {
+    } else if (warp == STAGER_WARP) {
         // ------------------------------------------------------------ outer-scale stager
         int ob = 0;
         uint32_t ophase = 0u;                         // bit b: phase of outer buffer b
@@ -226,12 +228,14 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ promotion + epilogue
+        constexpr int COLS = BN / 2;            // columns of this warp
         const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;
         int pb = 0, ob = 0;
         uint32_t pphase = 0u, ophase = 0u;            // bit b: phase of buffer b
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN;
+            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN + half * COLS;
             const int row = m0 + 32 * q + lane;
             int got = 0;
             if (lane == 0) {
@@ -239,10 +243,10 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 if (!got) raise_timeout(p, abort_flag);
             }
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
-            const float* outer_tile = outer_b + ob * (MAX_CHUNKS * BN);
-            float2 acc[BN / 2];
+            const float* outer_tile = outer_b + ob * (MAX_CHUNKS * BN) + half * COLS;
+            float2 acc[COLS / 2];
 #pragma unroll
-            for (int c = 0; c < BN / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
+            for (int c = 0; c < COLS / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
             const float* a_outer_row = p.a_outer + (int64_t)row * nkc;
             float sa_next = __ldg(a_outer_row);
             for (int kc = 0; kc < nkc; ++kc) {
@@ -258,41 +262,43 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     break;
                 }
                 sm100::tc_fence_after();
-                // acc += sa * (sB * P), 32 columns at a time, packed
-                const float2 sa2 = make_float2(sa, sa);
-                const float4* sb = reinterpret_cast<const float4*>(outer_tile + kc * BN);
+                // the whole slice in one burst, then release the buffer
+                uint32_t r[COLS];
 #pragma unroll
-                for (int c32 = 0; c32 < BN / 32; ++c32) {
-                    uint32_t r[32];
-                    sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + BN * pb + 32 * c32, r);
-                    sm100::tmem_ld_wait();
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float4 w = sb[8 * c32 + c];
-                        const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1])),
-                                                     make_float2(w.x, w.y));
-                        const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3])),
-                                                     make_float2(w.z, w.w));
-                        acc[16 * c32 + 2 * c] = __ffma2_rn(t0, sa2, acc[16 * c32 + 2 * c]);
-                        acc[16 * c32 + 2 * c + 1] = __ffma2_rn(t1, sa2, acc[16 * c32 + 2 * c + 1]);
-                    }
+                for (int c32 = 0; c32 < COLS / 32; ++c32) {
+                    uint32_t (&rr)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[32 * c32]);
+                    sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + BN * pb + half * COLS + 32 * c32, rr);
                 }
+                sm100::tmem_ld_wait();
                 sm100::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) sm100::mbar_arrive(&pempty[pb]);     // the tensor core may refill it
                 pphase ^= 1u << pb;
                 pb ^= 1;
+                // acc += sa * (sB * P), packed
+                const float2 sa2 = make_float2(sa, sa);
+                const float4* sb = reinterpret_cast<const float4*>(outer_tile + kc * BN);
+#pragma unroll
+                for (int c = 0; c < COLS / 4; ++c) {
+                    const float4 w = sb[c];
+                    const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1])),
+                                                 make_float2(w.x, w.y));
+                    const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3])),
+                                                 make_float2(w.z, w.w));
+                    acc[2 * c] = __ffma2_rn(t0, sa2, acc[2 * c]);
+                    acc[2 * c + 1] = __ffma2_rn(t1, sa2, acc[2 * c + 1]);
+                }
             }
             __syncwarp();
             if (lane == 0) sm100::mbar_arrive(&oempty[ob]);          // this tile's outer scales are used
             ophase ^= 1u << ob;
             ob ^= 1;
             if (!ok) break;
-            // store the tile's row
+            // store this warp's part of the tile's row
             if (OUT_BF16) {
                 uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + n0);
 #pragma unroll
-                for (int v = 0; v < BN / 8; ++v) {
+                for (int v = 0; v < COLS / 8; ++v) {
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -304,7 +310,7 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             } else {
                 float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)row * p.ldc + n0);
 #pragma unroll
-                for (int v = 0; v < BN / 4; ++v)
+                for (int v = 0; v < COLS / 4; ++v)
                     dst[v] = make_float4(acc[2 * v].x, acc[2 * v].y, acc[2 * v + 1].x, acc[2 * v + 1].y);
             }
         }

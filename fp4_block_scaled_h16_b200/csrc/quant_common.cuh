@@ -278,38 +278,37 @@ __device__ __forceinline__ void nv_divide(float* v, const float2* SY) {
 }
 
 // ------------------------------------------------------------------ encoders
-__device__ __forceinline__ uint32_t sign_nibbles8(const float* v) {
-    uint32_t s = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s |= (__float_as_uint(v[j]) >> 31) << (4 * j + 3);
-    return s;
-}
 
-__device__ __forceinline__ uint32_t sr_e2m1(float u, uint32_t r) {
-    u = fminf(u, 6.0f);
-    float lo, winv, base;
-    if (u < 2.0f) {
-        const float t = floorf(__fmul_rn(u, 2.0f));
-        base = t; lo = __fmul_rn(t, 0.5f); winv = 2.0f;
-    } else if (u < 4.0f) {
-        const float t = floorf(u);
-        base = __fadd_rn(t, 2.0f); lo = t; winv = 1.0f;
-    } else if (u < 6.0f) {
-        base = 6.0f; lo = 4.0f; winv = 0.5f;
+// Stochastic rounding of |v| onto E2M1, as an exact integer test: with lo the
+// level below u = min(|v|, 6), w the gap above it and t = (r >> 8) * 2^-24,
+// "round up iff t < (u - lo) / w" is "(r >> 8) < ceil(2^24 (u - lo) / w)".
+// For u >= 1 the levels are u's exponent with one mantissa bit, so lo clears
+// the low 22 mantissa bits and 2^24 (u - lo) / w is those bits times 4; on
+// [0.5, 1) lo = 0.5, w = 0.5 and it is the 23-bit mantissa times 2; below
+// 0.5 it is u * 2^25.  Returns the magnitude index.
+__device__ __forceinline__ uint32_t sr_e2m1(float v, uint32_t r) {
+    const float u = fminf(fabsf(v), 6.0f);
+    const uint32_t ub = __float_as_uint(u);
+    uint32_t lo_idx, F;
+    if (u >= 1.0f) {
+        lo_idx = (ub >> 22) - 252u;                // 1 -> 2, 1.5 -> 3, 2 -> 4, ... 6 -> 7
+        F = (ub & 0x3FFFFFu) << 2;
+    } else if (u >= 0.5f) {
+        lo_idx = 1u;
+        F = (ub & 0x7FFFFFu) << 1;
     } else {
-        base = 7.0f; lo = 6.0f; winv = 0.0f;
+        lo_idx = 0u;
+        F = __float2uint_ru(__fmul_rn(u, 0x1p25f));
     }
-    const float f = __fmul_rn(__fsub_rn(u, lo), winv);
-    const float t = __fmul_rn((float)(r >> 8), 0x1p-24f);
-    return (uint32_t)base + (t < f ? 1u : 0u);
+    return lo_idx + ((r >> 8) < F ? 1u : 0u);
 }
 
-__device__ __forceinline__ uint32_t sr_ufp4(float u, uint32_t r) {
-    u = fminf(u, 7.0f);
+// the same on the uniform grid k = 0..7: lo = floor(u), w = 1
+__device__ __forceinline__ uint32_t sr_ufp4(float v, uint32_t r) {
+    const float u = fminf(fabsf(v), 7.0f);
     const float t = floorf(u);
-    const float f = __fsub_rn(u, t);
-    const float th = __fmul_rn((float)(r >> 8), 0x1p-24f);
-    return (uint32_t)t + (th < f ? 1u : 0u);
+    const uint32_t F = __float2uint_ru(__fmul_rn(__fsub_rn(u, t), 0x1p24f));
+    return (uint32_t)t + ((r >> 8) < F ? 1u : 0u);
 }
 
 // 8 scaled values -> one word of codes, element j in nibble j
@@ -332,13 +331,13 @@ __device__ __forceinline__ uint32_t encode8(const float* v, const uint32_t* rnd)
     uint32_t w = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const float u = fabsf(v[j]);
         uint32_t k;
-        if (FMT == UFP4) k = SR ? sr_ufp4(u, rnd[j]) : (uint32_t)__float2int_rn(fminf(u, 7.0f));
-        else             k = sr_e2m1(u, rnd[j]);
-        w |= k << (4 * j);
+        if (FMT == UFP4) k = SR ? sr_ufp4(v[j], rnd[j]) : (uint32_t)__float2int_rn(fminf(fabsf(v[j]), 7.0f));
+        else             k = sr_e2m1(v[j], rnd[j]);
+        // magnitude and sign bit (bit 31 of v moved to bit 3 of the nibble)
+        w |= (k | ((__float_as_uint(v[j]) >> 28) & 8u)) << (4 * j);
     }
-    return w | sign_nibbles8(v);
+    return w;
 }
 
 // ------------------------------------------------------------------ division by a constant

@@ -132,16 +132,31 @@ quant_cols_kernel(const QuantArgs a) {
     for (int q = 0; q < 4; ++q) {
         uint32_t rnd[2][8];
         if (SR) {
-            // element (r, line): i = r * C + line.  With C % 4 == 0 the two
-            // lines of a row share one Philox group (words line0 % 4 and +1).
+            // element (r, line): i = r * C + line.  With C % 4 == 0 the four
+            // lines of lanes 2t and 2t+1 share one Philox group per row: each
+            // lane of the pair draws every other row and they swap two words.
+            if ((C & 3) == 0) {
+                const uint32_t par = lane & 1;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint64_t i = (uint64_t)(rbase + 8 * q + k) * (uint64_t)C + (uint64_t)line0;
-                const uint4 wds = sr_words(i >> 2, a.tensor_id, a.keys);
-                rnd[0][k] = word_of(wds, (int)(i & 3));
-                if ((C & 3) == 0) {
-                    rnd[1][k] = word_of(wds, (int)(i & 3) + 1);
-                } else {
+                for (int m = 0; m < 4; ++m) {
+                    const uint64_t row = (uint64_t)(rbase + 8 * q + 2 * m + par);
+                    const uint64_t i = row * (uint64_t)C + (uint64_t)(line0 - 2 * par);   // group start
+                    const uint4 wds = sr_words(i >> 2, a.tensor_id, a.keys);
+                    const uint32_t mine0 = par ? wds.z : wds.x, mine1 = par ? wds.w : wds.y;
+                    const uint32_t send0 = par ? wds.x : wds.z, send1 = par ? wds.y : wds.w;
+                    const uint32_t recv0 = __shfl_xor_sync(0xffffffffu, send0, 1);
+                    const uint32_t recv1 = __shfl_xor_sync(0xffffffffu, send1, 1);
+                    // row 2m is the even lane's, row 2m+1 the odd lane's
+                    rnd[0][2 * m] = par ? recv0 : mine0;
+                    rnd[1][2 * m] = par ? recv1 : mine1;
+                    rnd[0][2 * m + 1] = par ? mine0 : recv0;
+                    rnd[1][2 * m + 1] = par ? mine1 : recv1;
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t i = (uint64_t)(rbase + 8 * q + k) * (uint64_t)C + (uint64_t)line0;
+                    rnd[0][k] = word_of(sr_words(i >> 2, a.tensor_id, a.keys), (int)(i & 3));
                     const uint64_t i1 = i + 1;
                     rnd[1][k] = word_of(sr_words(i1 >> 2, a.tensor_id, a.keys), (int)(i1 & 3));
                 }
