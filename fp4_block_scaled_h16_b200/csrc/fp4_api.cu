@@ -267,7 +267,7 @@ fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
     if (double_block && (!a_outer || !b_outer)) return FP4_ERR_INVALID_ARG;
     const int64_t es = out_dtype == FP4_OUT_BF16 ? 2 : 4;
     if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
-        !aligned16(c) || (ldc * es) % 16)
+        !aligned16(c) || (ldc * es) % 16 || (double_block && (!aligned16(a_outer) || !aligned16(b_outer))))
         return FP4_ERR_MISALIGNED;
     int dev;
     fp4_status_t st;

@@ -7,11 +7,13 @@
 //
 // The outer scale changes every 128 elements of K, so it cannot ride in the
 // tensor core's E4M3 block scales.  Each 128-K chunk is two block-scaled MMAs
-// (tcgen05 kind::mxf4nvf4, 128 x 128 x 64) into one of two TMEM partial
-// buffers; while the tensor core fills one, the epilogue warps promote the
-// other: acc[i, j] += s_oA[i, kc] * (s_oB[j, kc] * P_kc[i, j]) in registers,
-// on packed f32x2 pairs.  The operand pipeline (TMA producer warp, MMA warp,
-// 4-stage ring of 256-K stages) is the one of the plain GEMM; a seventh warp
+// (tcgen05 kind::mxf4nvf4, 128 x 128 x 64) into one of three TMEM partial
+// buffers in rotation; while the tensor core fills one, sixteen epilogue
+// warps (four per TMEM lane quarter, so each scheduler has four to hide the
+// TMEM and shared-load latency) promote another:
+// acc[i, j] += s_oA[i, kc] * (s_oB[j, kc] * P_kc[i, j]) in registers, on
+// packed f32x2 pairs.  The operand pipeline (TMA producer warp, MMA warp,
+// 4-stage ring of 256-K stages) is the one of the plain GEMM; one more warp
 // stages each tile's B outer scales transposed ([chunk][column]) into a
 // double-buffered shared area, so the promotion reads four of them per
 // 128-bit shared load.  All hand-offs are mbarriers with bounded waits.
@@ -30,7 +32,9 @@ namespace {
 
 constexpr int BM = 128, BN = 128, BK = 256;
 constexpr int STAGES = 4;
-constexpr int EPI_WARPS = 8;              // two per TMEM lane quarter, half of the columns each
+constexpr int EPI_WARPS = 16;             // four per TMEM lane quarter, a quarter of the columns each
+constexpr int COLS = BN / (EPI_WARPS / 4);      // columns one epilogue warp promotes
+constexpr int HALF = COLS / 2;                  // columns per TMEM load
 constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS + 1);   // producer, MMA, epilogue, outer-scale warp
 constexpr int STAGER_WARP = 2 + EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
@@ -44,7 +48,8 @@ constexpr uint32_t TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr uint32_t STAGE_BYTES = (TX + 1023) / 1024 * 1024;
 constexpr uint32_t OUTER_BYTES = 2 * MAX_CHUNKS * BN * 4;   // s_oB of two tiles, [chunk][column]
 constexpr uint32_t SMEM = STAGES * STAGE_BYTES + OUTER_BYTES + 1024 + 256;
-constexpr uint32_t SFA_COL = 2 * BN;                  // TMEM: partials at 0 and BN, then scales
+constexpr int PBUF = 3;                               // TMEM partial buffers in rotation
+constexpr uint32_t SFA_COL = PBUF * BN;               // TMEM: partials at 0, BN, 2 BN, then scales
 constexpr uint32_t SFB_COL = SFA_COL + 16;
 
 struct DbParams {
@@ -76,8 +81,8 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + OUTER_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* pfull = empty + STAGES;          // partial buffer b holds a finished chunk
-    uint64_t* pempty = pfull + 2;              // partial buffer b was read by the epilogue
-    uint64_t* ofull = pempty + 2;              // outer-scale buffer b is staged for a tile
+    uint64_t* pempty = pfull + PBUF;           // partial buffer b was read by the epilogue
+    uint64_t* ofull = pempty + PBUF;           // outer-scale buffer b is staged for a tile
     uint64_t* oempty = ofull + 2;              // the epilogue is done with outer buffer b
     uint64_t* drain = oempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -89,9 +94,11 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             sm100::mbar_init(&full[s], 1);
             sm100::mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < PBUF; ++b) {
             sm100::mbar_init(&pfull[b], 1);
             sm100::mbar_init(&pempty[b], EPI_WARPS);
+        }
+        for (int b = 0; b < 2; ++b) {
             sm100::mbar_init(&ofull[b], 32);
             sm100::mbar_init(&oempty[b], EPI_WARPS);
         }
@@ -188,7 +195,7 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         issued = true;
                         sm100::tc_commit(&pfull[pb]);
                         pphase ^= 1u << pb;
-                        pb ^= 1;
+                        pb = (pb + 1 == PBUF) ? 0 : pb + 1;
                     }
                     if (!ok) break;
                     sm100::tc_commit(&empty[stage]);
@@ -213,13 +220,14 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 if (lane == 0) raise_timeout(p, abort_flag);
                 break;
             }
-            // rows n0 .. n0+127 of [N, K/128] are one contiguous run: read it
-            // coalesced, write it transposed
+            // rows n0 .. n0+127 of [N, K/128] (16 KB at most, L1-resident after
+            // the first chunk) written transposed; consecutive lanes take
+            // consecutive columns so the shared stores do not collide on a bank
             float* dst = outer_b + ob * (MAX_CHUNKS * BN);
             const float* src = p.b_outer + (int64_t)n0 * nkc;
             for (int e = lane; e < BN * nkc; e += 32) {
-                const int c = e / nkc, kc = e - c * nkc;
-                dst[kc * BN + c] = __ldg(src + e);
+                const int kc = e / BN, c = e % BN;
+                dst[e] = __ldg(src + c * nkc + kc);
             }
             __syncwarp();
             sm100::mbar_arrive(&ofull[ob]);          // release: every lane's stores before
@@ -228,66 +236,88 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ promotion + epilogue
-        constexpr int COLS = BN / 2;            // columns of this warp
         const int q = warp & 3;                 // TMEM lane quarter of this warp
-        const int half = (warp - 2) >> 2;
+        const int cg = (warp - 2) >> 2;         // column group of this warp
         int pb = 0, ob = 0;
         uint32_t pphase = 0u, ophase = 0u;            // bit b: phase of buffer b
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN + half * COLS;
+            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN + cg * COLS;
             const int row = m0 + 32 * q + lane;
-            int got = 0;
-            if (lane == 0) {
-                got = sm100::mbar_wait(&ofull[ob], (ophase >> ob) & 1u, p.wait_limit, abort_flag) ? 1 : 0;
-                if (!got) raise_timeout(p, abort_flag);
+            if (!__all_sync(0xffffffffu, sm100::mbar_wait(&ofull[ob], (ophase >> ob) & 1u, p.wait_limit, abort_flag))) {
+                if (lane == 0) raise_timeout(p, abort_flag);
+                break;
             }
-            if (!__shfl_sync(0xffffffffu, got, 0)) break;
-            const float* outer_tile = outer_b + ob * (MAX_CHUNKS * BN) + half * COLS;
+            const float* outer_tile = outer_b + ob * (MAX_CHUNKS * BN) + cg * COLS;
             float2 acc[COLS / 2];
 #pragma unroll
             for (int c = 0; c < COLS / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
-            const float* a_outer_row = p.a_outer + (int64_t)row * nkc;
-            float sa_next = __ldg(a_outer_row);
-            for (int kc = 0; kc < nkc; ++kc) {
-                const float sa = sa_next;
-                if (kc + 1 < nkc) sa_next = __ldg(a_outer_row + kc + 1);
-                got = 0;
-                if (lane == 0) {
-                    got = sm100::mbar_wait(&pfull[pb], (pphase >> pb) & 1u, p.wait_limit, abort_flag) ? 1 : 0;
-                    if (!got) raise_timeout(p, abort_flag);
-                }
-                if (!__shfl_sync(0xffffffffu, got, 0)) {
-                    ok = false;
-                    break;
-                }
+            // row outer scales two chunks at a time (K / 128 is even), one pair ahead
+            const float2* a_outer_row = reinterpret_cast<const float2*>(p.a_outer + (int64_t)row * nkc);
+            float2 sa_cur = __ldg(a_outer_row);
+            float2 sa_nxt = nkc > 2 ? __ldg(a_outer_row + 1) : sa_cur;
+            // the slice is read in two halves of 16 columns: one half's TMEM load
+            // is in flight while the other half is promoted
+            const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + cg * COLS;
+            uint32_t ra[HALF], rb[HALF];
+            if (!__all_sync(0xffffffffu, sm100::mbar_wait(&pfull[pb], (pphase >> pb) & 1u, p.wait_limit, abort_flag))) {
+                if (lane == 0) raise_timeout(p, abort_flag);
+                ok = false;
+            } else {
                 sm100::tc_fence_after();
-                // the whole slice in one burst, then release the buffer
-                uint32_t r[COLS];
-#pragma unroll
-                for (int c32 = 0; c32 < COLS / 32; ++c32) {
-                    uint32_t (&rr)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[32 * c32]);
-                    sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + BN * pb + half * COLS + 32 * c32, rr);
-                }
-                sm100::tmem_ld_wait();
-                sm100::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) sm100::mbar_arrive(&pempty[pb]);     // the tensor core may refill it
-                pphase ^= 1u << pb;
-                pb ^= 1;
-                // acc += sa * (sB * P), packed
+                sm100::tmem_ld16(tbase + BN * pb, ra);
+                sm100::tmem_ld_wait_on(ra);
+            }
+            for (int kc = 0; kc < nkc && ok; ++kc) {
+                const float sa = (kc & 1) ? sa_cur.y : sa_cur.x;
                 const float2 sa2 = make_float2(sa, sa);
                 const float4* sb = reinterpret_cast<const float4*>(outer_tile + kc * BN);
+                sm100::tmem_ld16(tbase + BN * pb + HALF, rb);
+                // acc += sa * (sB * P) on the first half, packed
 #pragma unroll
-                for (int c = 0; c < COLS / 4; ++c) {
+                for (int c = 0; c < HALF / 4; ++c) {
                     const float4 w = sb[c];
-                    const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1])),
+                    const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(ra[4 * c]), __uint_as_float(ra[4 * c + 1])),
                                                  make_float2(w.x, w.y));
-                    const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3])),
+                    const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(ra[4 * c + 2]), __uint_as_float(ra[4 * c + 3])),
                                                  make_float2(w.z, w.w));
                     acc[2 * c] = __ffma2_rn(t0, sa2, acc[2 * c]);
                     acc[2 * c + 1] = __ffma2_rn(t1, sa2, acc[2 * c + 1]);
                 }
+                sm100::tmem_ld_wait_on(rb);
+                sm100::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(&pempty[pb]);     // the tensor core may refill it
+                pphase ^= 1u << pb;
+                pb = (pb + 1 == PBUF) ? 0 : pb + 1;
+                if (kc & 1) {
+                    sa_cur = sa_nxt;
+                    if (kc + 3 < nkc) sa_nxt = __ldg(a_outer_row + (kc + 3) / 2);
+                }
+                bool next = false;
+                if (kc + 1 < nkc) {
+                    if (__all_sync(0xffffffffu,
+                                   sm100::mbar_wait(&pfull[pb], (pphase >> pb) & 1u, p.wait_limit, abort_flag))) {
+                        sm100::tc_fence_after();
+                        sm100::tmem_ld16(tbase + BN * pb, ra);
+                        next = true;
+                    } else {
+                        if (lane == 0) raise_timeout(p, abort_flag);
+                        ok = false;
+                    }
+                }
+                // the second half, while the next chunk's first half loads
+#pragma unroll
+                for (int c = 0; c < HALF / 4; ++c) {
+                    const float4 w = sb[HALF / 4 + c];
+                    const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(rb[4 * c]), __uint_as_float(rb[4 * c + 1])),
+                                                 make_float2(w.x, w.y));
+                    const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(rb[4 * c + 2]), __uint_as_float(rb[4 * c + 3])),
+                                                 make_float2(w.z, w.w));
+                    acc[HALF / 2 + 2 * c] = __ffma2_rn(t0, sa2, acc[HALF / 2 + 2 * c]);
+                    acc[HALF / 2 + 2 * c + 1] = __ffma2_rn(t1, sa2, acc[HALF / 2 + 2 * c + 1]);
+                }
+                if (next) sm100::tmem_ld_wait_on(ra);
             }
             __syncwarp();
             if (lane == 0) sm100::mbar_arrive(&oempty[ob]);          // this tile's outer scales are used

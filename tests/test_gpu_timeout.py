@@ -1,0 +1,59 @@
+"""Failure detection of the GEMM pipelines without a GPU fault.
+
+Every hand-off inside the GEMM kernels (TMA producer -> MMA issuer ->
+epilogue, and the double-block GEMM's partial and outer-scale buffers) is an
+mbarrier wait bounded by a poll limit.  When a wait runs out, the kernel
+raises an abort flag that the other roles see, lets its copies and MMAs in
+flight finish, frees TMEM and returns; the host learns of it through
+fp4_last_error as FP4_ERR_TIMEOUT.
+
+Here the limit is lowered to one poll (about a microsecond), far below the
+time a K = 8192 tile needs, so the first wait of the epilogue runs out.  The
+test checks the status, and that the context is still usable: the next call
+with the default limit gives the same bits as a call made before the timeout,
+and reports FP4_OK.
+"""
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp4(cuda_device):
+    from fp4_block_scaled_h16_b200 import fp4 as m
+    return m
+
+
+def operands(fp4, fmt, double_block, M=256, N=256, K=8192, seed=5):
+    g = torch.Generator().manual_seed(seed)
+    a = torch.randn((M, K), generator=g).to(torch.bfloat16).cuda()
+    b = torch.randn((N, K), generator=g).to(torch.bfloat16).cuda()
+    kw = dict(fmt=fmt, double_block=double_block, axis=1)
+    return fp4.quantize(a, tensor_id=1, **kw), fp4.quantize(b, tensor_id=2, **kw)
+
+
+@pytest.mark.parametrize("fmt,double_block,out", [
+    ("MXFP4", False, "F32"),
+    ("NVFP4", False, "BF16"),
+    ("NVFP4", True, "BF16"),
+    ("NVFP4", True, "F32"),
+])
+def test_gemm_wait_timeout_is_reported_and_recoverable(fp4, fmt, double_block, out):
+    qa, qb = operands(fp4, getattr(fp4, "FP4_" + fmt), double_block)
+    out_dtype = getattr(fp4, "FP4_OUT_" + out)
+    before = fp4.gemm(qa, qb, out_dtype)
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+
+    fp4.fp4_set_wait_limit(1)
+    try:
+        fp4.gemm(qa, qb, out_dtype)
+        status = fp4.fp4_last_error()
+    finally:
+        fp4.fp4_set_wait_limit(0)
+    assert status == fp4.FP4_ERR_TIMEOUT, fp4.fp4_status_string(status)
+
+    after = fp4.gemm(qa, qb, out_dtype)
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    assert torch.equal(before.view(torch.int16 if out == "BF16" else torch.int32),
+                       after.view(torch.int16 if out == "BF16" else torch.int32))
