@@ -233,10 +233,17 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
     const int rn = rot_size(rotation);
     const bool bf16 = in_dtype == FP4_IN_BF16;
     if (internal_amax) {
-        if (cudaMemsetAsync(workspace, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
+        // workspace words: 0 the amax (binary32 bits), 1 the grid-barrier count
+        if (cudaMemsetAsync(workspace, 0, 2 * sizeof(unsigned int), s) != cudaSuccess) return FP4_ERR_CUDA;
         a.amax_out = static_cast<unsigned int*>(workspace);
-        if (launch_amax(a, bf16, rn, axis, s) != cudaSuccess) return FP4_ERR_CUDA;
+        a.grid_count = static_cast<unsigned int*>(workspace) + 1;
         a.amax_in = static_cast<const float*>(workspace);
+        if (axis == 1) {
+            // one launch: amax pass, grid barrier, quantize pass
+            if (launch_quantize_fused(a, bf16, format, rounding == FP4_SR, rn, s) != cudaSuccess) return FP4_ERR_CUDA;
+            return FP4_OK;
+        }
+        if (launch_amax(a, bf16, rn, axis, s) != cudaSuccess) return FP4_ERR_CUDA;
     } else {
         a.amax_in = tensor_amax;
     }

@@ -20,6 +20,7 @@ struct QuantArgs {
     float* tensor_scale_out;
     const float* amax_in;       // rotated-tensor amax (NVFP4 / UFP4 without double block)
     unsigned int* amax_out;     // amax pass: atomicMax target (binary32 bits, >= 0)
+    unsigned int* grid_count;   // fused launch: arrivals at the grid barrier (zeroed by the host)
     PhiloxKeys keys;
     uint32_t tensor_id;
     uint32_t sign_mask;         // random-sign bits (0: deterministic Hadamard)
@@ -30,6 +31,9 @@ struct QuantArgs {
 cudaError_t launch_quantize(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, bool db, int axis,
                             cudaStream_t s);
 cudaError_t launch_amax(QuantArgs a, bool bf16, int rot_n, int axis, cudaStream_t s);
+// NVFP4 / UFP4, row axis: amax pass, grid barrier and quantize pass in one
+// cooperative launch; a.amax_out / a.grid_count point at zeroed words
+cudaError_t launch_quantize_fused(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, cudaStream_t s);
 cudaError_t launch_quantize_cols(const QuantArgs& a, bool bf16, int fmt, bool sr, int rot_n, bool signs,
                                  bool db, cudaStream_t s);
 cudaError_t launch_amax_cols(const QuantArgs& a, bool bf16, int rot_n, bool signs, cudaStream_t s);

@@ -233,6 +233,31 @@ __device__ __forceinline__ uint32_t block_scale_code(float m, const ScaleRef& re
     return cvt_e4m3(sb);
 }
 
+// the codes of NB blocks with maxima m[]: one test for the whole unit decides
+// whether every division is in the range where the reciprocal-and-correction
+// form is exact (a zero maximum passes: it gives code 0 either way), and the
+// common case then runs without branches; otherwise block_scale_code per block
+template <int FMT, int NB>
+__device__ __forceinline__ void block_scale_codes(const float* m, const ScaleRef& ref, uint32_t* code) {
+    constexpr float Q = (FMT == UFP4) ? 7.0f : 6.0f;
+    constexpr float YQ = (FMT == UFP4) ? 0x1.24924ap-3f : 0x1.555556p-3f;   // RN(1/7), RN(1/6)
+    float n[NB];
+    bool fast = ref.fast;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        n[b] = div_rcp(m[b], Q, YQ);
+        const bool in_range = m[b] >= 0x1p-122f && n[b] >= 0x1p-100f && __fmul_rn(n[b], ref.y) < 0x1p100f;
+        fast = fast && (m[b] == 0.0f || in_range);
+    }
+    if (fast) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) code[b] = cvt_e4m3(div_rcp(n[b], ref.s, ref.y));
+    } else {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) code[b] = block_scale_code<FMT>(m[b], ref);
+    }
+}
+
 // S = RN(E * s_ref) and y = RN(1/S) for block scale code E; y = 0 marks a
 // block that takes the slow path: IEEE division when S or 1/S is outside the
 // normal range, and, for E = 0 (S = 0), x * 0, the signed zeros of the codes.
@@ -257,6 +282,25 @@ struct ScaleTable {
 template <int U, int ROT>
 __device__ __forceinline__ void nv_divide(float* v, const float2* SY) {
     using PL = PairLayout<U, ROT>;
+    bool slow = false;
+#pragma unroll
+    for (int b = 0; b < U / 16; ++b) slow = slow || SY[b].y == 0.0f;
+    if (!slow) {
+        // every block of the unit on the exact reciprocal path: no branches
+#pragma unroll
+        for (int p = 0; p < PL::N; ++p) {
+            const int j = PL::lo(p), k = j + PL::PS;
+            const float2 a = SY[j / 16], b = SY[k / 16];
+            const float2 x = make_float2(v[j], v[k]);
+            const float2 yy = make_float2(a.y, b.y);
+            const float2 q0 = mul2(x, yy);
+            const float2 r = __ffma2_rn(make_float2(-a.x, -b.x), q0, x);
+            const float2 q = __ffma2_rn(r, yy, q0);
+            v[j] = q.x;
+            v[k] = q.y;
+        }
+        return;
+    }
 #pragma unroll
     for (int p = 0; p < PL::N; ++p) {
         const int j = PL::lo(p), k = j + PL::PS;

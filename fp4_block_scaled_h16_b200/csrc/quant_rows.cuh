@@ -18,126 +18,213 @@ namespace fp4 {
 
 constexpr int RQ_THREADS = 256;
 constexpr uint32_t RQ_WAIT_LIMIT = 1u << 24;
+constexpr uint32_t RQ_GRID_WAIT_LIMIT = 1u << 22;   // polls of the grid barrier (32 ns sleeps)
 
-// a stage holds one U-element unit per thread; 3 stages (2 for 32-KB stages)
-template <bool BF16, int U>
+// what a launch does: quantize with a known tensor amax, compute the rotated
+// tensor's amax only, or both in one launch (amax pass, grid barrier, quantize pass)
+enum RowMode { RQ_QUANT = 0, RQ_AMAX = 1, RQ_FUSED = 2 };
+
+// CTAs per SM that registers allow without spills (the SR variants carry a
+// Philox word per element)
+template <bool SR, int MODE>
+constexpr int row_ctas_by_regs() { return MODE == RQ_AMAX ? 4 : (SR ? 2 : 3); }
+
+// A stage holds one U-element unit per thread; the ring has 3 stages (2 when
+// the SM's CTAs cannot hold 3), two of them loading while one is computed.
+// (Measured on B200: refilling the previous stage's slot from one thread
+// beats refilling each slot the moment its last warp has copied it out, and
+// a fourth stage adds nothing.)
+template <bool BF16, int U, bool SR, int MODE>
 struct RowRing {
     static constexpr int BYTES = RQ_THREADS * U * (BF16 ? 2 : 4);
-    static constexpr int STAGES = BYTES <= 16384 ? 3 : 2;
-    static constexpr int SMEM = STAGES * BYTES + STAGES * 8;
+    static constexpr int FIT = (200 * 1024) / (row_ctas_by_regs<SR, MODE>() * BYTES);
+    static constexpr int STAGES = FIT < 3 ? 2 : 3;
+    static constexpr int SMEM = STAGES * BYTES + STAGES * 16;   // + a full and an empty barrier per stage
 };
 
-// CTAs per SM: as many as registers allow without spills (the SR variants
-// carry a Philox word per element) and shared memory allows
-template <bool BF16, int U, bool SR, bool AMAX_ONLY>
+// CTAs per SM: what registers and shared memory both allow
+template <bool BF16, int U, bool SR, int MODE>
 constexpr int row_ctas() {
-    constexpr int by_smem = (228 * 1024) / (RowRing<BF16, U>::SMEM + 1024 + 2048);
-    constexpr int by_regs = AMAX_ONLY ? 4 : (SR ? 2 : 3);
+    constexpr int by_smem = (228 * 1024) / (RowRing<BF16, U, SR, MODE>::SMEM + 1024 + 2048);
+    constexpr int by_regs = row_ctas_by_regs<SR, MODE>();
     return by_smem < by_regs ? by_smem : by_regs;
 }
 
 struct RowStages {
-    int64_t total;          // number of stages
-    int64_t lps;            // lines per stage (>= 1) when a line fits, else 0
-    int64_t segs;           // segments per line when it does not (else 1)
-    int64_t seg_elems;      // elements per segment
+    int total;              // number of stages (< 2^31)
+    int lps;                // lines per stage (>= 1) when a line fits, else 0
+    int segs;               // segments per line when it does not (else 1)
+    int seg_elems;          // elements per segment
     uint32_t seg_m, seg_l;  // multiply-shift division by segs
 };
 
-template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY, int U>
-__global__ void __launch_bounds__(RQ_THREADS, (row_ctas<BF16, U, SR, AMAX_ONLY>()))
+template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE, int U>
+__global__ void __launch_bounds__(RQ_THREADS, (row_ctas<BF16, U, SR, MODE>()))
 quant_rows_kernel(const QuantArgs a, const RowStages st) {
     static_assert(U == 16 || U == 32, "unit size");
+    constexpr bool AMAX_ONLY = MODE == RQ_AMAX, FUSED = MODE == RQ_FUSED;
+    static_assert(!FUSED || (FMT != MXFP4 && !DB), "only a tensor-scaled format has an amax pass");
     constexpr int ES = BF16 ? 2 : 4;
     constexpr int CHUNKS = U * ES / 16;                 // 16-byte chunks per unit
-    using Ring = RowRing<BF16, U>;
+    using Ring = RowRing<BF16, U, SR, MODE>;
     constexpr int RQ_STAGES = Ring::STAGES, RQ_STAGE_BYTES = Ring::BYTES;
+    constexpr int WARPS = RQ_THREADS / 32;
     extern __shared__ __align__(128) uint8_t rq_smem[];
     uint8_t* buf = rq_smem;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(rq_smem + RQ_STAGES * RQ_STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(rq_smem + RQ_STAGES * RQ_STAGE_BYTES);  // stage landed
+    uint64_t* empty = full + RQ_STAGES;                 // every warp has copied the stage out
     const int tid = threadIdx.x, lane = tid & 31;
 
     __shared__ ScaleTable table;                        // (S, 1/S) per E4M3 code under s_t
     ScaleRef ref_t = make_ref(1.0f);
-    if (!AMAX_ONLY && FMT != MXFP4 && !DB) {
+    __shared__ float warp_max[RQ_THREADS / 32];          // FUSED: the amax pass's result
+    __shared__ uint32_t grid_verdict;
+    if (MODE == RQ_QUANT && FMT != MXFP4 && !DB) {
         ref_t = make_ref(tensor_scale_of(*a.amax_in, FMT));
         if (blockIdx.x == 0 && tid == 0 && a.tensor_scale_out) *a.tensor_scale_out = ref_t.s;
         table.build(ref_t.s, tid, RQ_THREADS);
     }
     if (tid == 0) {
-        for (int s = 0; s < RQ_STAGES; ++s) sm100::mbar_init(&bar[s], 1);
+        for (int s = 0; s < RQ_STAGES; ++s) {
+            sm100::mbar_init(&full[s], 1);
+            sm100::mbar_init(&empty[s], WARPS);
+        }
         sm100::fence_barrier_init();
     }
     __syncthreads();
 
-    // stage s -> its first line, line count and element range
-    auto stage_geom = [&](int64_t s, int64_t& l0, int64_t& nl, int64_t& e0, int64_t& ne) {
+    // stage s -> its first line, line count and element range (all below 2^31:
+    // the launcher checks the stage count, and K and the lines per stage are
+    // bounded by it)
+    auto stage_geom = [&](int s, int& l0, int& nl, int& e0, int& ne) {
         if (st.lps) {
             l0 = s * st.lps;
-            nl = min(st.lps, a.L - l0);
+            nl = min(st.lps, (int)(a.L - l0));
             e0 = 0;
-            ne = a.K;
+            ne = (int)a.K;
         } else {
-            l0 = fast_div((uint32_t)s, st.seg_m, st.seg_l);
+            l0 = (int)fast_div((uint32_t)s, st.seg_m, st.seg_l);
             nl = 1;
             e0 = (s - l0 * st.segs) * st.seg_elems;
-            ne = min(st.seg_elems, a.K - e0);
+            ne = min(st.seg_elems, (int)(a.K - e0));
         }
     };
     // one thread fills a stage buffer: one bulk copy per line piece
-    auto issue = [&](int64_t s, int slot) {
-        int64_t l0, nl, e0, ne;
+    auto issue = [&](int s, int slot) {
+        int l0, nl, e0, ne;
         stage_geom(s, l0, nl, e0, ne);
         const uint32_t bytes = (uint32_t)(ne * ES);
-        sm100::mbar_arrive_expect_tx(&bar[slot], bytes * (uint32_t)nl);
-        for (int64_t r = 0; r < nl; ++r) {
-            const uint8_t* src = static_cast<const uint8_t*>(a.x) + ((l0 + r) * a.ld + e0) * ES;
-            sm100::bulk_load(buf + slot * RQ_STAGE_BYTES + r * bytes, src, bytes, &bar[slot]);
+        sm100::mbar_arrive_expect_tx(&full[slot], bytes * (uint32_t)nl);
+        for (int r = 0; r < nl; ++r) {
+            const uint8_t* src = static_cast<const uint8_t*>(a.x) + ((int64_t)(l0 + r) * a.ld + e0) * ES;
+            sm100::bulk_load(buf + slot * RQ_STAGE_BYTES + r * bytes, src, bytes, &full[slot]);
         }
     };
 
-    const int64_t first = blockIdx.x, stride = gridDim.x;
+    // this CTA's stages first, first + stride, ... (n of them) make one pass;
+    // a fused launch streams them twice through the ring, the second pass in
+    // reverse order so that the most recently read stages, the likeliest to
+    // be still in L2, come first
+    const int first = blockIdx.x, stride = gridDim.x;
+    const int n = first < st.total ? (st.total - first + stride - 1) / stride : 0;
+    const int nv = FUSED ? 2 * n : n;
+    auto stage_of = [&](int v) { return (FUSED && v >= n) ? first + (2 * n - 1 - v) * stride : first + v * stride; };
     if (tid == 0)
         for (int p = 0; p < RQ_STAGES - 1; ++p)
-            if (first + p * stride < st.total) issue(first + p * stride, p);
+            if (p < nv) issue(stage_of(p), p);
 
     // this thread's unit within a full stage: line my_li of the stage, unit my_ju
-    const int64_t full_nl = st.lps ? st.lps : 1;
-    const int64_t full_ne = st.lps ? a.K : st.seg_elems;
-    const int64_t my_li = st.lps > 1 ? (int64_t)fast_div((uint32_t)tid, a.div_m, a.div_l) : 0;
-    const int64_t my_ju = tid - my_li * (full_ne / U);
-    const bool my_active = (int64_t)tid < full_nl * (full_ne / U);
+    const int full_nl = st.lps ? st.lps : 1;
+    const int full_ne = st.lps ? (int)a.K : st.seg_elems;
+    const int my_li = st.lps > 1 ? (int)fast_div((uint32_t)tid, a.div_m, a.div_l) : 0;
+    const int my_ju = tid - my_li * (full_ne / U);
+    const bool my_active = tid < full_nl * (full_ne / U);
 
     float tmax = 0.0f;
     bool ok = true;
-    int it = 0;
-    for (int64_t s = first; s < st.total; s += stride, ++it) {
+    for (int it = 0; it < nv; ++it) {
+        if (FUSED && it == n) {
+            // end of the amax pass: the CTA's maximum, then the grid's, then
+            // the tensor scale and its table.  Every thread of the CTA gets
+            // here (a failed wait of the first pass skips to this point).
+            const uint32_t wbits = __reduce_max_sync(0xffffffffu, __float_as_uint(tmax));
+            if (lane == 0) warp_max[tid >> 5] = __uint_as_float(wbits);
+            const bool failed = __syncthreads_or(!ok);
+            if (tid == 0) {
+                float m = 0.0f;
+#pragma unroll
+                for (int w = 0; w < RQ_THREADS / 32; ++w) m = fmaxf(m, warp_max[w]);
+                if (__float_as_uint(m)) atomicMax(a.amax_out, __float_as_uint(m));
+                __threadfence();
+                atomicAdd(a.grid_count, 1u);
+                bool done = false;
+                for (uint32_t i = 0; i < RQ_GRID_WAIT_LIMIT; ++i) {
+                    if (sm100::ld_acquire_gpu(a.grid_count) >= gridDim.x) { done = true; break; }
+                    __nanosleep(32);
+                }
+                if (!done) atomicExch(a.err, 7u);       // FP4_ERR_TIMEOUT
+                warp_max[0] = __uint_as_float(sm100::ld_acquire_gpu(a.amax_out));
+                grid_verdict = (done && !failed) ? 1u : 0u;
+            }
+            __syncthreads();
+            if (!grid_verdict) {
+                ok = false;
+                break;
+            }
+            ref_t = make_ref(tensor_scale_of(warp_max[0], FMT));
+            if (blockIdx.x == 0 && tid == 0 && a.tensor_scale_out) *a.tensor_scale_out = ref_t.s;
+            table.build(ref_t.s, tid, RQ_THREADS);
+            __syncthreads();
+        }
+        const int s = stage_of(it);
         const int slot = it % RQ_STAGES;
-        const bool got = sm100::mbar_wait(&bar[slot], (uint32_t)(it / RQ_STAGES) & 1u, RQ_WAIT_LIMIT, nullptr);
-        // one barrier per stage: the verdict is the CTA's, and every thread is
-        // done with the previous stage's slot, which is refilled next
-        if (__syncthreads_or(!got)) {
-            ok = false;                               // a copy that never lands: stop, report
+        // the verdict on a wait is the warp's; a copy that never lands stops
+        // the warp (in the first pass of a fused launch: sends it on to the
+        // pass boundary, where the whole CTA meets)
+        if (!__all_sync(0xffffffffu,
+                        sm100::mbar_wait(&full[slot], (uint32_t)(it / RQ_STAGES) & 1u, RQ_WAIT_LIMIT, nullptr))) {
+            ok = false;
+            if (FUSED && it < n) { it = n - 1; continue; }
             break;
         }
-        if (tid == 0 && s + (RQ_STAGES - 1) * stride < st.total)
-            issue(s + (RQ_STAGES - 1) * stride, (it + RQ_STAGES - 1) % RQ_STAGES);
-
-        int64_t l0, nl, e0, ne;
+        int l0, nl, e0, ne;
         stage_geom(s, l0, nl, e0, ne);
-        const bool active = (nl == full_nl && ne == full_ne) ? my_active : (int64_t)tid < nl * (ne / U);
+        const bool active = (nl == full_nl && ne == full_ne) ? my_active : tid < nl * (ne / U);
         const int64_t l = l0 + my_li;
         const int64_t j = e0 / U + my_ju;             // unit index within the line
 
-        // read the unit from shared memory (128-bit loads; the 4-way bank
+        // copy the unit out of shared memory (128-bit loads; the 4-way bank
         // conflicts of the 64-byte unit stride still leave shared memory far
-        // faster than HBM)
-        float v[U];
+        // faster than HBM), then release the slot: the warps run on without
+        // waiting for one another, and only the refilling thread waits, for
+        // the copies of the previous stage, long done by then
+        uint4 w[CHUNKS];
         if (active) {
             const uint4* src = reinterpret_cast<const uint4*>(buf + slot * RQ_STAGE_BYTES + (my_li * ne + my_ju * U) * ES);
-            uint4 w[CHUNKS];
 #pragma unroll
             for (int q = 0; q < CHUNKS; ++q) w[q] = src[q];
+        }
+        // the warp's copies are done: release the slot; thread 0 refills the
+        // previous stage's slot, which every warp released long ago
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&empty[slot]);
+        bool stalled = false;
+        if (tid == 0 && it + RQ_STAGES - 1 < nv) {
+            const int refill = (it + RQ_STAGES - 1) % RQ_STAGES;
+            if (it > 0 && !sm100::mbar_wait(&empty[refill], (uint32_t)((it - 1) / RQ_STAGES) & 1u,
+                                            RQ_WAIT_LIMIT, nullptr))
+                stalled = true;
+            else
+                issue(stage_of(it + RQ_STAGES - 1), refill);
+        }
+        if (__any_sync(0xffffffffu, stalled)) {
+            ok = false;
+            if (FUSED && it < n) { it = n - 1; continue; }
+            break;
+        }
+
+        float v[U];
+        if (active) {
 #pragma unroll
             for (int q = 0; q < CHUNKS; ++q) {
                 if (BF16) {
@@ -154,7 +241,7 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
 #pragma unroll
             for (int e = 0; e < U; ++e) v[e] = 0.0f;
         }
-        if (AMAX_ONLY) {
+        if (AMAX_ONLY || (FUSED && it < n)) {
             tmax = unit_rotated_absmax<U, ROT, SIGNS>(v, a.sign_mask, tmax);
             continue;
         }
@@ -176,11 +263,12 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
                 if (active && (lane & (GL - 1)) == 0) a.outer[l * (a.K / 128) + (j * U) / 128] = ref.s;
             }
             float2 SY[U / 16];
+            float bm[U / 16];
 #pragma unroll
-            for (int b = 0; b < U / 16; ++b) {
-                sbytes[b] = block_scale_code<FMT>(absmax_n<16>(v + 16 * b), ref);
-                SY[b] = DB ? scale_pair(sbytes[b], ref.s) : table.e[sbytes[b]];
-            }
+            for (int b = 0; b < U / 16; ++b) bm[b] = absmax_n<16>(v + 16 * b);
+            block_scale_codes<FMT, U / 16>(bm, ref, sbytes);
+#pragma unroll
+            for (int b = 0; b < U / 16; ++b) SY[b] = DB ? scale_pair(sbytes[b], ref.s) : table.e[sbytes[b]];
             nv_divide<U, ROT>(v, SY);
         }
         if (!active) continue;
@@ -215,7 +303,7 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
     }
 
     if (!ok) {
-        if (tid == 0) atomicExch(a.err, 7u);          // FP4_ERR_TIMEOUT
+        if (lane == 0) atomicExch(a.err, 7u);         // FP4_ERR_TIMEOUT
         return;
     }
     if (AMAX_ONLY) {
@@ -224,69 +312,95 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
     }
 }
 
-template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY, int U>
+template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE, int U>
 cudaError_t launch_rows(const QuantArgs& a, cudaStream_t s) {
     constexpr int ES = BF16 ? 2 : 4;
-    using Ring = RowRing<BF16, U>;
+    using Ring = RowRing<BF16, U, SR, MODE>;
+    auto kernel = quant_rows_kernel<BF16, FMT, SR, ROT, SIGNS, DB, MODE, U>;
     static bool attr_set = false;   // per instantiation
+    static int resident = 0;        // CTAs per SM the launch can keep resident
     if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(quant_rows_kernel<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY, U>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, Ring::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Ring::SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, RQ_THREADS, Ring::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
+    // stage, line and element indices inside the kernel are 32-bit
+    if (a.L >= ((int64_t)1 << 31) || a.K >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     RowStages st{};
     const int64_t line_bytes = a.K * ES;
+    int64_t total;
     if (line_bytes <= Ring::BYTES) {
-        st.lps = Ring::BYTES / line_bytes;            // whole lines, one unit per thread at most
-        st.total = (a.L + st.lps - 1) / st.lps;
+        st.lps = (int)(Ring::BYTES / line_bytes);     // whole lines, one unit per thread at most
+        total = (a.L + st.lps - 1) / st.lps;
         st.segs = 1;
-        st.seg_elems = a.K;
+        st.seg_elems = (int)a.K;
     } else {
         st.lps = 0;
-        st.seg_elems = (int64_t)RQ_THREADS * U;       // a multiple of 128 elements
-        st.segs = (a.K + st.seg_elems - 1) / st.seg_elems;
-        st.total = a.L * st.segs;
+        st.seg_elems = RQ_THREADS * U;                // a multiple of 128 elements
+        st.segs = (int)((a.K + st.seg_elems - 1) / st.seg_elems);
+        total = a.L * st.segs;
     }
-    if (st.total >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;   // stage indices are 32-bit
+    if (total >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    st.total = (int)total;
     uint32_t l = 0;
     while (l < 32 && (uint64_t(1) << l) < (uint64_t)st.segs) ++l;
     st.seg_m = (uint32_t)((uint64_t)(((unsigned __int128)1 << (32 + l)) / (uint64_t)st.segs) - (uint64_t(1) << 32) + 1);
     st.seg_l = l;
-    int64_t grid = (int64_t)num_sms() * row_ctas<BF16, U, SR, AMAX_ONLY>();
-    if (grid > st.total) grid = st.total;
+    const int per_sm = resident < row_ctas<BF16, U, SR, MODE>() ? resident : row_ctas<BF16, U, SR, MODE>();
+    int64_t grid = (int64_t)num_sms() * (per_sm > 0 ? per_sm : 1);
+    if (grid > total) grid = total;
     if (grid < 1) grid = 1;
-    quant_rows_kernel<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY, U><<<(unsigned)grid, RQ_THREADS, Ring::SMEM, s>>>(a, st);
+    if (MODE == RQ_FUSED) {
+        // the grid barrier between the passes needs every CTA resident at once
+        if (resident < 1) return cudaErrorInvalidConfiguration;
+        QuantArgs ka = a;
+        RowStages kst = st;
+        void* args[] = {&ka, &kst};
+        return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3((unsigned)grid),
+                                           dim3(RQ_THREADS), args, Ring::SMEM, s);
+    }
+    kernel<<<(unsigned)grid, RQ_THREADS, Ring::SMEM, s>>>(a, st);
     return cudaGetLastError();
 }
 
 // unit size: 32 when the line length allows it (always for MXFP4 and 32-rotations)
-template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY>
+template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE>
 cudaError_t rows_by_unit(const QuantArgs& a, cudaStream_t s) {
     if (FMT == MXFP4 || ROT == 32 || DB || a.K % 32 == 0)
-        return launch_rows<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY, 32>(a, s);
-    return launch_rows<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY, (FMT == MXFP4 || ROT == 32 || DB) ? 32 : 16>(a, s);
+        return launch_rows<BF16, FMT, SR, ROT, SIGNS, DB, MODE, 32>(a, s);
+    return launch_rows<BF16, FMT, SR, ROT, SIGNS, DB, MODE, (FMT == MXFP4 || ROT == 32 || DB) ? 32 : 16>(a, s);
 }
 
-template <bool BF16, int FMT, bool SR, bool DB, bool AMAX_ONLY>
+template <bool BF16, int FMT, bool SR, bool DB, int MODE>
 cudaError_t rows_by_rot(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s) {
-    if (rot_n == 0) return rows_by_unit<BF16, FMT, SR, 0, false, DB, AMAX_ONLY>(a, s);
-    if (rot_n == 16) return signs ? rows_by_unit<BF16, FMT, SR, 16, true, DB, AMAX_ONLY>(a, s)
-                                  : rows_by_unit<BF16, FMT, SR, 16, false, DB, AMAX_ONLY>(a, s);
-    return signs ? rows_by_unit<BF16, FMT, SR, 32, true, DB, AMAX_ONLY>(a, s)
-                 : rows_by_unit<BF16, FMT, SR, 32, false, DB, AMAX_ONLY>(a, s);
+    if (rot_n == 0) return rows_by_unit<BF16, FMT, SR, 0, false, DB, MODE>(a, s);
+    if (rot_n == 16) return signs ? rows_by_unit<BF16, FMT, SR, 16, true, DB, MODE>(a, s)
+                                  : rows_by_unit<BF16, FMT, SR, 16, false, DB, MODE>(a, s);
+    return signs ? rows_by_unit<BF16, FMT, SR, 32, true, DB, MODE>(a, s)
+                 : rows_by_unit<BF16, FMT, SR, 32, false, DB, MODE>(a, s);
 }
 
 template <bool BF16>
 cudaError_t rows_by_fmt(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db, cudaStream_t s) {
-    if (fmt == MXFP4) return sr ? rows_by_rot<BF16, MXFP4, true, false, false>(a, rot_n, signs, s)
-                                : rows_by_rot<BF16, MXFP4, false, false, false>(a, rot_n, signs, s);
-    if (fmt == UFP4) return sr ? rows_by_rot<BF16, UFP4, true, false, false>(a, rot_n, signs, s)
-                               : rows_by_rot<BF16, UFP4, false, false, false>(a, rot_n, signs, s);
-    if (db) return sr ? rows_by_rot<BF16, NVFP4, true, true, false>(a, rot_n, signs, s)
-                      : rows_by_rot<BF16, NVFP4, false, true, false>(a, rot_n, signs, s);
-    return sr ? rows_by_rot<BF16, NVFP4, true, false, false>(a, rot_n, signs, s)
-              : rows_by_rot<BF16, NVFP4, false, false, false>(a, rot_n, signs, s);
+    if (fmt == MXFP4) return sr ? rows_by_rot<BF16, MXFP4, true, false, RQ_QUANT>(a, rot_n, signs, s)
+                                : rows_by_rot<BF16, MXFP4, false, false, RQ_QUANT>(a, rot_n, signs, s);
+    if (fmt == UFP4) return sr ? rows_by_rot<BF16, UFP4, true, false, RQ_QUANT>(a, rot_n, signs, s)
+                               : rows_by_rot<BF16, UFP4, false, false, RQ_QUANT>(a, rot_n, signs, s);
+    if (db) return sr ? rows_by_rot<BF16, NVFP4, true, true, RQ_QUANT>(a, rot_n, signs, s)
+                      : rows_by_rot<BF16, NVFP4, false, true, RQ_QUANT>(a, rot_n, signs, s);
+    return sr ? rows_by_rot<BF16, NVFP4, true, false, RQ_QUANT>(a, rot_n, signs, s)
+              : rows_by_rot<BF16, NVFP4, false, false, RQ_QUANT>(a, rot_n, signs, s);
+}
+
+// NVFP4 / UFP4 with the tensor amax computed in the same launch
+template <bool BF16>
+cudaError_t rows_fused_by_fmt(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, cudaStream_t s) {
+    if (fmt == UFP4) return sr ? rows_by_rot<BF16, UFP4, true, false, RQ_FUSED>(a, rot_n, signs, s)
+                               : rows_by_rot<BF16, UFP4, false, false, RQ_FUSED>(a, rot_n, signs, s);
+    return sr ? rows_by_rot<BF16, NVFP4, true, false, RQ_FUSED>(a, rot_n, signs, s)
+              : rows_by_rot<BF16, NVFP4, false, false, RQ_FUSED>(a, rot_n, signs, s);
 }
 
 // one input type's entry points (defined in quantize.cu for bf16, quantize_rows_f32.cu for f32)
@@ -298,7 +412,12 @@ cudaError_t launch_rows_quantize(const QuantArgs& a, int fmt, bool sr, int rot_n
 
 template <bool BF16>
 cudaError_t launch_rows_amax(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s) {
-    return rows_by_rot<BF16, NVFP4, false, false, true>(a, rot_n, signs, s);
+    return rows_by_rot<BF16, NVFP4, false, false, RQ_AMAX>(a, rot_n, signs, s);
+}
+
+template <bool BF16>
+cudaError_t launch_rows_fused(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, cudaStream_t s) {
+    return rows_fused_by_fmt<BF16>(a, fmt, sr, rot_n, signs, s);
 }
 
 }  // namespace fp4

@@ -25,6 +25,7 @@ namespace fp4 {
 
 extern template cudaError_t launch_rows_quantize<false>(const QuantArgs&, int, bool, int, bool, bool, cudaStream_t);
 extern template cudaError_t launch_rows_amax<false>(const QuantArgs&, int, bool, cudaStream_t);
+extern template cudaError_t launch_rows_fused<false>(const QuantArgs&, int, bool, int, bool, cudaStream_t);
 
 namespace {
 
@@ -50,6 +51,13 @@ cudaError_t launch_quantize(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n,
     set_divisor(a, (uint32_t)(a.K / unit_of(fmt, rot_n, a.K)));
     return bf16 ? launch_rows_quantize<true>(a, fmt, sr, rot_n, signs, db, s)
                 : launch_rows_quantize<false>(a, fmt, sr, rot_n, signs, db, s);
+}
+
+cudaError_t launch_quantize_fused(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, cudaStream_t s) {
+    const bool signs = a.sign_mask != 0u;
+    set_divisor(a, (uint32_t)(a.K / unit_of(fmt, rot_n, a.K)));
+    return bf16 ? launch_rows_fused<true>(a, fmt, sr, rot_n, signs, s)
+                : launch_rows_fused<false>(a, fmt, sr, rot_n, signs, s);
 }
 
 cudaError_t launch_amax(QuantArgs a, bool bf16, int rot_n, int axis, cudaStream_t s) {

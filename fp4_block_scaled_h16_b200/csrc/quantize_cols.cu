@@ -118,11 +118,12 @@ quant_cols_kernel(const QuantArgs a) {
             sbytes[cc][1] = 1u;
         } else {
             float2 SY[2];
+            float bm[2];
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                sbytes[cc][b] = block_scale_code<FMT>(absmax_n<16>(v[cc] + 16 * b), s_ref[cc]);
-                SY[b] = DB ? scale_pair(sbytes[cc][b], s_ref[cc].s) : table.e[sbytes[cc][b]];
-            }
+            for (int b = 0; b < 2; ++b) bm[b] = absmax_n<16>(v[cc] + 16 * b);
+            block_scale_codes<FMT, 2>(bm, s_ref[cc], sbytes[cc]);
+#pragma unroll
+            for (int b = 0; b < 2; ++b) SY[b] = DB ? scale_pair(sbytes[cc][b], s_ref[cc].s) : table.e[sbytes[cc][b]];
             nv_divide<32, ROT>(v[cc], SY);
         }
     }

@@ -6,7 +6,8 @@
 // inside a CUDA-graph capture that must not allocate, in a plug-in whose host
 // framework owns every device allocation, or in a real-time loop that may not
 // touch the allocator.  Such callers still own their inputs and outputs; only
-// the 4-byte amax accumulator moves into library-owned memory.
+// the scratch words (the amax accumulator and a grid-barrier count) move into
+// library-owned memory.
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <mutex>
@@ -15,8 +16,9 @@
 
 namespace {
 
-// One FP32 slot is used (the rotated-tensor amax); the array is sized like
-// the workspace fp4_quantize requests, 256 bytes.  Every GPU that loads the
+// Two 32-bit words are used (the rotated-tensor amax and a grid-barrier
+// count); the array is sized like the workspace fp4_quantize requests, 256
+// bytes.  Every GPU that loads the
 // library holds one copy until the process exits.
 constexpr size_t kScratchBytes = 256;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -62,8 +64,8 @@ extern "C" fp4_status_t fp4_quantize_noalloc(const void* x, fp4_in_dtype_t in_dt
     fp4_status_t st = fp4_quantize_workspace_size(format, 0, 0, &need);
     if (st != FP4_OK) return st;
     if (need > kScratchBytes) return FP4_ERR_WORKSPACE;    // larger than the static array
-    // check what fp4_quantize would reject before anything is launched;
-    // fp4_amax below checks the input itself and launches nothing on error
+    // check what fp4_quantize would reject before anything is launched (it
+    // checks the input itself and launches nothing on error)
     if (rounding != FP4_RTNE && rounding != FP4_SR) return FP4_ERR_INVALID_ARG;
     if (axis != 0 && axis != 1) return FP4_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0) return FP4_ERR_INVALID_ARG;
@@ -80,10 +82,9 @@ extern "C" fp4_status_t fp4_quantize_noalloc(const void* x, fp4_in_dtype_t in_dt
         return fp4_quantize(x, in_dtype, rows, cols, ld, format, rounding, rotation, axis, 0, seed,
                             tensor_id, amax, codes, scales, nullptr, tensor_scale, nullptr, 0, stream);
     }
-    // fp4_amax clears the slot (it must start at zero) and accumulates the
-    // rotated-tensor amax into it; fp4_quantize then builds s_t from it
-    st = fp4_amax(x, in_dtype, rows, cols, ld, rotation, axis, seed, amax, stream);
-    if (st != FP4_OK) return st;
+    // the static array is the workspace of fp4_quantize's internal amax: it
+    // clears it on the stream, then accumulates the rotated-tensor amax (and,
+    // on the row axis, the grid-barrier count of its one-launch path) there
     return fp4_quantize(x, in_dtype, rows, cols, ld, format, rounding, rotation, axis, 0, seed, tensor_id,
-                        amax, codes, scales, nullptr, tensor_scale, nullptr, 0, stream);
+                        nullptr, codes, scales, nullptr, tensor_scale, scratch, kScratchBytes, stream);
 }

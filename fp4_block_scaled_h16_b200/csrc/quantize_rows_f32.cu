@@ -6,5 +6,6 @@ namespace fp4 {
 
 template cudaError_t launch_rows_quantize<false>(const QuantArgs&, int, bool, int, bool, bool, cudaStream_t);
 template cudaError_t launch_rows_amax<false>(const QuantArgs&, int, bool, cudaStream_t);
+template cudaError_t launch_rows_fused<false>(const QuantArgs&, int, bool, int, bool, cudaStream_t);
 
 }  // namespace fp4

@@ -156,7 +156,11 @@ fp4_status_t fp4_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int6
  *   seed, tensor_id SR stream and random signs (tensor_id only for SR)
  *   tensor_amax     optional device float: the rotated-tensor amax to build
  *                   s_t from (e.g. the max over shards); NULL = computed here,
- *                   which needs the workspace
+ *                   which needs the workspace.  On the row axis (axis = 1)
+ *                   the amax pass and the quantize pass then run as one
+ *                   cooperative launch whose CTAs meet at a grid barrier (the
+ *                   second read of x mostly hits L2); on axis 0 they are two
+ *                   launches
  *   codes           device uint8 [L, K/2]
  *   scales          device, fp4_scales_bytes(L, K, format) bytes, tiled layout
  *   outer_scales    device float [L, K/128] (double block), else ignored
@@ -183,8 +187,9 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
  * fp4_quantize asks for.  The pages have no counterpart to this call; it only
  * changes where the scratch lives.
  *
- * The scratch is a static device array of 256 bytes inside libfp4.so (one
- * FP32 amax slot is used); every GPU that loads the library holds one copy
+ * The scratch is a static device array of 256 bytes inside libfp4.so (two
+ * 32-bit words are used: the amax and a grid-barrier count); every GPU that
+ * loads the library holds one copy
  * until the process exits.  A request needing more scratch than that returns
  * FP4_ERR_WORKSPACE (every NVFP4 / UFP4 shape needs exactly the 256 bytes).
  * The caller still owns x, codes, scales and tensor_scale, with the layouts,
@@ -195,8 +200,8 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
  * The first call on a device resolves the array's device address on that
  * device (cudaGetSymbolAddress), so make it before any stream capture.  Every
  * call shares the one array and leaves its amax there; each call clears the
- * slot before accumulating into it.  Calls that overlap on the GPU (other
- * streams, other threads, concurrent graph launches) race on the slot and
+ * words before accumulating into them.  Calls that overlap on the GPU (other
+ * streams, other threads, concurrent graph launches) race on them and
  * must be serialized by the caller.  Allocates nothing; errors as
  * fp4_quantize, checked before anything is launched.
  */

@@ -184,3 +184,29 @@ def test_layer_linear_operands(fp4, name, fmt):
         kw = dict(fmt=fmt, rounding=sr, rotation=1, axis=axis, seed=0, tensor_id=16 + role)
         g = gpu_quantize(fp4, d[t].cuda(), **kw)
         assert_quant_equal(g, oracle_quantize(d[t], **kw), what="%s %s %s" % (name, t, kw))
+
+
+# The internal amax on the row axis runs as one cooperative launch (amax pass,
+# grid barrier, quantize pass); it must give exactly what the two-launch path
+# gives: fp4_amax, then fp4_quantize with that amax.  The shapes cover fewer
+# stages than CTAs, many lines per stage, a ragged last stage and lines split
+# into segments (a line longer than one stage).
+@pytest.mark.parametrize("shape", [(1, 16), (3, 48), (257, 4096), (1000, 272), (9, 24576)])
+@pytest.mark.parametrize("fmt,rounding,rot", [(NV, 0, 1), (NV, 1, 4), (UF, 0, 0), (UF, 1, 3)])
+def test_one_launch_amax_matches_two_launches(fp4, shape, fmt, rounding, rot):
+    R, C = shape
+    if C % (32 if rot in (2, 4) else 16):
+        pytest.skip("rotation size does not divide the line")
+    x = make_input(R, C, "bf16", seed=R + C, outliers=R >= 2).cuda()
+    kw = dict(fmt=fmt, rounding=rounding, rotation=rot, axis=1, seed=11, tensor_id=3)
+    one, two = (fp4.alloc_qtensor(R, C, fmt, device=x.device) for _ in range(2))
+    for q in (one, two):
+        q["scales"].zero_()           # the tiled layout's padding is never written
+    fp4.quantize(x, out=one, **kw)
+    amax = torch.zeros(1, dtype=torch.float32, device=x.device)
+    fp4.fp4_amax(x, fp4.FP4_IN_BF16, R, C, C, rot, 1, 11, amax)
+    fp4.quantize(x, tensor_amax=amax, out=two, **kw)
+    torch.cuda.synchronize()
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    for key in ("codes", "scales", "tensor_scale"):
+        assert torch.equal(one[key].view(torch.uint8), two[key].view(torch.uint8)), key
