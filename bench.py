@@ -36,6 +36,11 @@ M, N, K = workloads.TOKENS, workloads.QKV_OUT, workloads.HIDDEN
 WORKLOAD = "nvfp4_fprop_qkv_%dx%dx%d" % (M, N, K)
 GEMM_FLOP = 2.0 * M * N * K
 L2_FLUSH_BYTES = 256 << 20
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gemm_kernel
+# launch on this workload, from one ncu capture of the current kernel: 36.4 MB
+# read (the 33 MB of operands cross DRAM once) and 49.7 MB written (the rest of
+# the 100.7 MB of C was still in L2 when the kernel ended)
+GEMM_TRAFFIC_BYTES = 36_395_520 + 49_682_944
 
 
 class L2Flush:
@@ -262,7 +267,8 @@ def run_gpu(args, rank, world, device):
                    "parallelism": "independent problem per GPU" if world > 1 else "single GPU"},
         "roofline": {"bound": "tensor", "kernel": "gemm_kernel (NVFP4, 128x256 tile)",
                      "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / fp4_peak, 4), "traffic": None,
+                     "frac": round(achieved / fp4_peak, 4), "traffic": GEMM_TRAFFIC_BYTES,
+                     "traffic_is": "ncu dram read + write bytes of one launch (algorithmic: 33.0 MB read, 100.7 MB written)",
                      "peak_is": "%s bf16 burst %.1f TFLOP/s x 4 (nominal fp4/bf16)" % (peaks["src"], peaks["bf16"])},
         "components": comp,
         "e2e": {"value": round(world * GEMM_FLOP / (e2e_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
@@ -299,9 +305,13 @@ def _qbytes(x, fmt, db):
     return n * x.element_size() + n / 2 + n / blk + (n / 128 * 4 if db else 0)
 
 
-def measure_configs(fp4, device, peaks, reps=10):
-    """Per-kernel timings of every workload: quantize GB/s and GEMM TFLOP/s with
-    their fractions of the measured HBM and derived FP4 peaks."""
+CONFIG_NAMES = ("tiny", "wgrad", "dgrad_db", "layer")
+
+
+def measure_configs(fp4, device, peaks, reps=10, only=CONFIG_NAMES):
+    """Per-kernel timings of every workload (or of those named in `only`):
+    quantize GB/s and GEMM TFLOP/s with their fractions of the measured HBM
+    and derived FP4 peaks."""
     flush = L2Flush(device)
     fp4_peak = peaks["bf16"] * 4.0
     out = {}
@@ -327,28 +337,35 @@ def measure_configs(fp4, device, peaks, reps=10):
     NV, MX, UF = fp4.FP4_NVFP4, fp4.FP4_MXFP4, fp4.FP4_UFP4
     BF, F32 = fp4.FP4_OUT_BF16, fp4.FP4_OUT_F32
 
-    d = workloads.tiny_mxfp4()
-    A, B = d["A"].to(device), d["B"].to(device)
-    qa, ea = quant_entry(A, fmt=MX, axis=1)
-    qb, eb = quant_entry(B, fmt=MX, axis=0)
-    out["tiny_mxfp4_256x256x512"] = {"quantize_A": ea, "quantize_B": eb, "gemm": gemm_entry(qa, qb, F32),
-                                     "note": "launch-bound; outside the roofline targets"}
+    if "tiny" in only:
+        d = workloads.tiny_mxfp4()
+        A, B = d["A"].to(device), d["B"].to(device)
+        qa, ea = quant_entry(A, fmt=MX, axis=1)
+        qb, eb = quant_entry(B, fmt=MX, axis=0)
+        out["tiny_mxfp4_256x256x512"] = {"quantize_A": ea, "quantize_B": eb, "gemm": gemm_entry(qa, qb, F32),
+                                         "note": "launch-bound; outside the roofline targets"}
 
-    d = workloads.mxfp4_wgrad_down()
-    dY, H = d["dY"].to(device), d["H"].to(device)
-    kw = dict(fmt=MX, rounding=fp4.FP4_SR, rotation=fp4.FP4_ROT_RH32, axis=0, seed=0)
-    qa, ea = quant_entry(dY, tensor_id=1, **kw)
-    qb, eb = quant_entry(H, tensor_id=2, **kw)
-    out["mxfp4_wgrad_down_4096x14336x8192"] = {"quantize_dY": ea, "quantize_H": eb, "gemm": gemm_entry(qa, qb, F32)}
-    del dY, H, qa, qb
+    if "wgrad" in only:
+        d = workloads.mxfp4_wgrad_down()
+        dY, H = d["dY"].to(device), d["H"].to(device)
+        kw = dict(fmt=MX, rounding=fp4.FP4_SR, rotation=fp4.FP4_ROT_RH32, axis=0, seed=0)
+        qa, ea = quant_entry(dY, tensor_id=1, **kw)
+        qb, eb = quant_entry(H, tensor_id=2, **kw)
+        out["mxfp4_wgrad_down_4096x14336x8192"] = {"quantize_dY": ea, "quantize_H": eb,
+                                                   "gemm": gemm_entry(qa, qb, F32)}
+        del dY, H, qa, qb
 
-    d = workloads.nvfp4_dgrad_down()
-    dY, Wd = d["dY"].to(device), d["Wd"].to(device)
-    kw = dict(fmt=NV, rounding=fp4.FP4_SR, double_block=True, seed=0)
-    qa, ea = quant_entry(dY, axis=1, tensor_id=1, **kw)
-    qb, eb = quant_entry(Wd, axis=0, tensor_id=2, **kw)
-    out["nvfp4_dgrad_down_db_8192x14336x4096"] = {"quantize_dY": ea, "quantize_Wd": eb, "gemm": gemm_entry(qa, qb, BF)}
-    del dY, Wd, qa, qb
+    if "dgrad_db" in only:
+        d = workloads.nvfp4_dgrad_down()
+        dY, Wd = d["dY"].to(device), d["Wd"].to(device)
+        kw = dict(fmt=NV, rounding=fp4.FP4_SR, double_block=True, seed=0)
+        qa, ea = quant_entry(dY, axis=1, tensor_id=1, **kw)
+        qb, eb = quant_entry(Wd, axis=0, tensor_id=2, **kw)
+        out["nvfp4_dgrad_down_db_8192x14336x4096"] = {"quantize_dY": ea, "quantize_Wd": eb,
+                                                      "gemm": gemm_entry(qa, qb, BF)}
+        del dY, Wd, qa, qb
+    if "layer" not in only:
+        return out
 
     # the decoder layer: Fprop, Dgrad, Wgrad of each linear in NVFP4 with H16
     # (SR on the Wgrad operands), then the UFP4 quantizer on the same operands
@@ -462,6 +479,8 @@ def main():
     ap.add_argument("--impl", choices=["fp4", "reference"], default="fp4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel table")
+    ap.add_argument("--configs", default=",".join(CONFIG_NAMES),
+                    help="comma-separated workloads of the per-config table: " + ", ".join(CONFIG_NAMES))
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -484,7 +503,11 @@ def main():
     if rank == 0:
         if world == 1 and not args.no_configs:
             from fp4_block_scaled_h16_b200 import fp4 as _fp4
-            line["configs"] = measure_configs(_fp4, device, measured_peaks())
+            only = tuple(c for c in args.configs.split(",") if c)
+            unknown = [c for c in only if c not in CONFIG_NAMES]
+            if unknown:
+                raise SystemExit("unknown --configs entries: %s" % ", ".join(unknown))
+            line["configs"] = measure_configs(_fp4, device, measured_peaks(), only=only)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(workloads.nvfp4_fprop_qkv(seed=0))
         print(json.dumps(line), flush=True)
