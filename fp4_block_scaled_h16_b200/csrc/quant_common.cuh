@@ -278,7 +278,8 @@ struct ScaleTable {
 
 // v <- v / S per element, S and y per 16-block (SY[b] = (S_b, y_b)), on the
 // unit's pair layout: q0 = x*y, r = x - S*q0 (exact), q = q0 + r*y = RN(x/S)
-// while S and 1/S are normal; IEEE division otherwise; S = y = 0 -> +-0.
+// while S and 1/S are normal (r is formed as -(S*q0 - x) so that x = -0
+// gives -0); IEEE division otherwise; S = y = 0 -> +-0.
 template <int U, int ROT>
 __device__ __forceinline__ void nv_divide(float* v, const float2* SY) {
     using PL = PairLayout<U, ROT>;
@@ -286,7 +287,10 @@ __device__ __forceinline__ void nv_divide(float* v, const float2* SY) {
 #pragma unroll
     for (int b = 0; b < U / 16; ++b) slow = slow || SY[b].y == 0.0f;
     if (!slow) {
-        // every block of the unit on the exact reciprocal path: no branches
+        // every block of the unit on the exact reciprocal path: no branches.
+        // The residual is taken as -(S q0 - x): the same value for x != 0, and
+        // for x = -0 it keeps q = -0 (x - S q0 would give +0 and lose the
+        // sign that the zero code carries)
 #pragma unroll
         for (int p = 0; p < PL::N; ++p) {
             const int j = PL::lo(p), k = j + PL::PS;
@@ -294,8 +298,8 @@ __device__ __forceinline__ void nv_divide(float* v, const float2* SY) {
             const float2 x = make_float2(v[j], v[k]);
             const float2 yy = make_float2(a.y, b.y);
             const float2 q0 = mul2(x, yy);
-            const float2 r = __ffma2_rn(make_float2(-a.x, -b.x), q0, x);
-            const float2 q = __ffma2_rn(r, yy, q0);
+            const float2 rn = __ffma2_rn(make_float2(a.x, b.x), q0, make_float2(-x.x, -x.y));
+            const float2 q = __ffma2_rn(make_float2(-rn.x, -rn.y), yy, q0);
             v[j] = q.x;
             v[k] = q.y;
         }
@@ -310,8 +314,8 @@ __device__ __forceinline__ void nv_divide(float* v, const float2* SY) {
             const float2 x = make_float2(v[j], v[k]);
             const float2 yy = make_float2(a.y, b.y);
             const float2 q0 = mul2(x, yy);
-            const float2 r = __ffma2_rn(make_float2(-a.x, -b.x), q0, x);
-            const float2 q = __ffma2_rn(r, yy, q0);
+            const float2 rn = __ffma2_rn(make_float2(a.x, b.x), q0, make_float2(-x.x, -x.y));   // -(x - S q0)
+            const float2 q = __ffma2_rn(make_float2(-rn.x, -rn.y), yy, q0);
             v[j] = q.x;
             v[k] = q.y;
         } else {

@@ -78,6 +78,8 @@ def special_values(R, C, seed):
     x[8, :] = np.float32(2.0 ** -149)
     x[9, :] = -1e-30
     x[9, 0] = 1.0                          # small negatives rounding to zero keep their sign
+    x[10, :] = -0.0
+    x[10, ::5] = rng.standard_normal(len(x[10, ::5]))   # -0 inside blocks with a nonzero maximum
     return torch.from_numpy(x)
 
 
