@@ -252,6 +252,87 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
     return FP4_OK;
 }
 
+fp4_status_t fp4_requantize(const uint8_t* src_codes, const uint8_t* src_scales, const float* src_outer,
+                            const float* src_tensor_scale, int64_t lines, int64_t K, fp4_format_t src_format,
+                            int src_double_block, fp4_format_t format, fp4_rounding_t rounding,
+                            fp4_rotation_t rotation, int double_block, uint64_t seed, uint32_t tensor_id,
+                            const float* tensor_amax, uint8_t* codes, uint8_t* scales, float* outer_scales,
+                            float* tensor_scale, void* workspace, size_t workspace_bytes, void* stream) {
+    // the source: `lines` lines of K elements (the rows of X^ [lines, K])
+    if (src_format < FP4_MXFP4 || src_format > FP4_UFP4) return FP4_ERR_INVALID_ARG;
+    if (src_double_block != 0 && src_double_block != 1) return FP4_ERR_INVALID_ARG;
+    if (src_double_block && src_format != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+    // the result: X^ quantized along axis 0, i.e. K lines of `lines` elements
+    if (format < FP4_MXFP4 || format > FP4_UFP4) return FP4_ERR_INVALID_ARG;
+    if (rounding != FP4_RTNE && rounding != FP4_SR) return FP4_ERR_INVALID_ARG;
+    if (rotation < FP4_ROT_NONE || rotation > FP4_ROT_RH32) return FP4_ERR_INVALID_ARG;
+    if (double_block != 0 && double_block != 1) return FP4_ERR_INVALID_ARG;
+    if (double_block && format != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+    if (lines < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    const bool empty = (lines == 0 || K == 0);
+    const int64_t sblk = (src_format == FP4_MXFP4) ? 32 : 16;
+    if (K % 16 || K % sblk || (src_double_block && K % 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    const int64_t blk = (format == FP4_MXFP4) ? 32 : 16;
+    const int rn = rot_size(rotation);
+    if (lines % blk || (rn && lines % rn) || (double_block && lines % 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    const bool src_ts = src_format != FP4_MXFP4 && !src_double_block;
+    const bool needs_ts = format != FP4_MXFP4 && !double_block;
+    const bool internal_amax = needs_ts && tensor_amax == nullptr;
+    if (!empty) {
+        if (!src_codes || !src_scales || (src_double_block && !src_outer) || (src_ts && !src_tensor_scale))
+            return FP4_ERR_INVALID_ARG;
+        if (!codes || !scales || (double_block && !outer_scales)) return FP4_ERR_INVALID_ARG;
+        if (!aligned16(src_codes) || !aligned16(codes)) return FP4_ERR_MISALIGNED;
+    }
+    if (needs_ts && !tensor_scale) return FP4_ERR_INVALID_ARG;
+    if ((src_outer && ((uintptr_t)src_outer & 3u)) || (src_tensor_scale && ((uintptr_t)src_tensor_scale & 3u)) ||
+        (outer_scales && ((uintptr_t)outer_scales & 3u)) || (tensor_scale && ((uintptr_t)tensor_scale & 3u)) ||
+        (tensor_amax && ((uintptr_t)tensor_amax & 3u)))
+        return FP4_ERR_MISALIGNED;
+    if (internal_amax && !empty) {
+        if (!workspace || workspace_bytes < 256) return FP4_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    }
+    int dev;
+    fp4_status_t st;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (empty) {
+        if (needs_ts) {
+            static const float one = 1.0f;
+            if (cudaMemcpyAsync(tensor_scale, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return FP4_ERR_CUDA;
+        }
+        return FP4_OK;
+    }
+    QuantArgs a{};
+    a.x = nullptr; a.rows = lines; a.cols = K; a.ld = K;
+    a.L = K; a.K = lines;
+    a.nb4 = ((lines / blk) + 3) / 4;
+    a.codes = codes; a.scales = scales; a.outer = outer_scales;
+    a.tensor_scale_out = needs_ts ? tensor_scale : nullptr;
+    a.keys = make_keys(seed);
+    a.tensor_id = tensor_id;
+    a.sign_mask = sign_mask_of(rotation, seed);
+    a.err = device_error_word();
+    a.src_codes = src_codes; a.src_scales = src_scales; a.src_outer = src_outer;
+    a.src_ts = src_tensor_scale;
+    a.src_fmt = src_format; a.src_db = src_double_block;
+    a.src_nb4 = ((K / sblk) + 3) / 4;
+    if (internal_amax) {
+        if (cudaMemsetAsync(workspace, 0, 2 * sizeof(unsigned int), s) != cudaSuccess) return FP4_ERR_CUDA;
+        a.amax_out = static_cast<unsigned int*>(workspace);
+        if (launch_requant_amax_cols(a, rn, a.sign_mask != 0u, s) != cudaSuccess) return FP4_ERR_CUDA;
+        a.amax_in = static_cast<const float*>(workspace);
+    } else {
+        a.amax_in = tensor_amax;
+    }
+    if (launch_requantize_cols(a, format, rounding == FP4_SR, rn, a.sign_mask != 0u, double_block != 0, s) !=
+        cudaSuccess)
+        return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
 fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
                       const uint8_t* a_codes, const uint8_t* a_scales, const float* a_outer,
                       const float* a_tensor_scale,

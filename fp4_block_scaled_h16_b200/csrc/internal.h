@@ -26,6 +26,14 @@ struct QuantArgs {
     uint32_t sign_mask;         // random-sign bits (0: deterministic Hadamard)
     uint32_t div_m, div_l;      // multiply-shift division by the units per line
     unsigned int* err;          // device error word (a bounded wait that ran out)
+    // re-quantization (fp4_requantize): the source is a quantized tensor whose
+    // lines are the rows of the logical [rows, cols] input; x is unused
+    const uint8_t* src_codes;   // [rows, cols/2]
+    const uint8_t* src_scales;  // tiled layout, src_nb4 groups of 4 blocks per line
+    const float* src_outer;     // [rows, cols/128] (double block)
+    const float* src_ts;        // tensor scale (NVFP4 / UFP4 without double block)
+    int src_fmt, src_db;
+    int64_t src_nb4;
 };
 
 cudaError_t launch_quantize(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, bool db, int axis,
@@ -37,6 +45,10 @@ cudaError_t launch_quantize_fused(QuantArgs a, bool bf16, int fmt, bool sr, int 
 cudaError_t launch_quantize_cols(const QuantArgs& a, bool bf16, int fmt, bool sr, int rot_n, bool signs,
                                  bool db, cudaStream_t s);
 cudaError_t launch_amax_cols(const QuantArgs& a, bool bf16, int rot_n, bool signs, cudaStream_t s);
+// the same two along axis 0 of the dequantized source (a.src_*)
+cudaError_t launch_requantize_cols(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db,
+                                   cudaStream_t s);
+cudaError_t launch_requant_amax_cols(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s);
 
 // GEMM
 struct GemmArgs {

@@ -14,7 +14,16 @@ namespace fp4 {
 // 32-element piece of two output lines, stored as 16 contiguous bytes each.
 constexpr int T0_ROWS = 128, T0_COLS = 64, T0_THREADS = 128;
 
-template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY>
+// one FP4 code of the source -> its grid value (E2M1 {0, .5, 1, 1.5, 2, 3, 4, 6}
+// or the UFP4 level k), sign from bit 3 (code 8 is -0)
+__device__ __forceinline__ float fp4_code_value(uint32_t n, bool ufp4) {
+    const uint32_t m = n & 7u;
+    const float mag = ufp4 ? (float)m : (float)((0xC8643210u >> (4u * m)) & 0xFu) * 0.5f;   // twice the level
+    return (n & 8u) ? -mag : mag;
+}
+
+// FP4SRC: the tile is the dequantized source X^ (fp4_requantize) instead of x
+template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY, bool FP4SRC = false>
 __global__ void __launch_bounds__(T0_THREADS)
 quant_cols_kernel(const QuantArgs a) {
     __shared__ __align__(16) float tile[T0_ROWS][T0_COLS + 4];
@@ -31,6 +40,46 @@ quant_cols_kernel(const QuantArgs a) {
         table.build(ref_t.s, tid, T0_THREADS);
     }
 
+    if constexpr (FP4SRC) {
+        // ---- stage the dequantized tile: one 16-element piece (8 bytes of
+        // codes, one block scale) per step, 4 per thread; zero outside [R, C).
+        // Element value: RN((q * E) * s_ref), where q * E is exact in binary32
+        // (E4M3 E, s_ref the tensor or outer scale); MXFP4: q * 2^(e - 127),
+        // exact (E = 1, s_ref = 2^(e - 127)).  C % 16 == 0, so pieces are whole.
+        const int sblk = a.src_fmt == MXFP4 ? 32 : 16;
+        const bool ufp4 = a.src_fmt == UFP4;
+        const float ts = (a.src_fmt != MXFP4 && !a.src_db) ? *a.src_ts : 1.0f;
+#pragma unroll
+        for (int it = 0; it < (T0_ROWS * T0_COLS / 16) / T0_THREADS; ++it) {
+            const int q = tid + it * T0_THREADS;
+            const int r = q >> 2, c = (q & 3) * 16;
+            const int64_t gr = row0 + r, gc = col0 + c;
+            float x[16];
+            if (gr < R && gc < C) {
+                const uint2 cw = __ldg(reinterpret_cast<const uint2*>(a.src_codes + gr * (C / 2) + gc / 2));
+                const uint32_t sb = a.src_scales[sf_offset(gr, gc / sblk, a.src_nb4)];
+                float E, s_ref;
+                if (a.src_fmt == MXFP4) {
+                    E = 1.0f;
+                    s_ref = sb ? __uint_as_float(sb << 23) : __uint_as_float(0x00400000u);   // 2^(sb - 127)
+                } else {
+                    E = e4m3_to_f32(sb);
+                    s_ref = a.src_db ? __ldg(a.src_outer + gr * (C / 128) + gc / 128) : ts;
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const uint32_t n = ((k < 8 ? cw.x : cw.y) >> (4 * (k & 7))) & 0xFu;
+                    x[k] = __fmul_rn(__fmul_rn(fp4_code_value(n, ufp4), E), s_ref);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) x[k] = 0.0f;
+            }
+#pragma unroll
+            for (int k = 0; k < 16; k += 4)
+                *reinterpret_cast<float4*>(&tile[r][c + k]) = make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
+        }
+    } else {
     // ---- stage the tile: 16-byte chunks, all loads issued first; zero outside [R, C)
     constexpr int EPC = BF16 ? 8 : 4;                    // elements per 16-byte chunk
     constexpr int CHUNKS = T0_ROWS * (T0_COLS / EPC);
@@ -71,6 +120,7 @@ quant_cols_kernel(const QuantArgs a) {
             *reinterpret_cast<float4*>(&tile[r][c]) = make_float4(__uint_as_float(raw[it].x), __uint_as_float(raw[it].y),
                                                                   __uint_as_float(raw[it].z), __uint_as_float(raw[it].w));
         }
+    }
     }
     __syncthreads();
 
@@ -189,32 +239,32 @@ quant_cols_kernel(const QuantArgs a) {
 
 namespace {
 
-template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY>
+template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY, bool FP4SRC>
 cudaError_t launch_cols(const QuantArgs& a, cudaStream_t s) {
     dim3 grid((unsigned)((a.cols + T0_COLS - 1) / T0_COLS), (unsigned)((a.rows + T0_ROWS - 1) / T0_ROWS));
-    quant_cols_kernel<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY><<<grid, T0_THREADS, 0, s>>>(a);
+    quant_cols_kernel<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY, FP4SRC><<<grid, T0_THREADS, 0, s>>>(a);
     return cudaGetLastError();
 }
 
-template <bool BF16, int FMT, bool SR, bool DB, bool AMAX_ONLY>
+template <bool BF16, int FMT, bool SR, bool DB, bool AMAX_ONLY, bool FP4SRC = false>
 cudaError_t cols_by_rot(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s) {
-    if (rot_n == 0) return launch_cols<BF16, FMT, SR, 0, false, DB, AMAX_ONLY>(a, s);
-    if (rot_n == 16) return signs ? launch_cols<BF16, FMT, SR, 16, true, DB, AMAX_ONLY>(a, s)
-                                  : launch_cols<BF16, FMT, SR, 16, false, DB, AMAX_ONLY>(a, s);
-    return signs ? launch_cols<BF16, FMT, SR, 32, true, DB, AMAX_ONLY>(a, s)
-                 : launch_cols<BF16, FMT, SR, 32, false, DB, AMAX_ONLY>(a, s);
+    if (rot_n == 0) return launch_cols<BF16, FMT, SR, 0, false, DB, AMAX_ONLY, FP4SRC>(a, s);
+    if (rot_n == 16) return signs ? launch_cols<BF16, FMT, SR, 16, true, DB, AMAX_ONLY, FP4SRC>(a, s)
+                                  : launch_cols<BF16, FMT, SR, 16, false, DB, AMAX_ONLY, FP4SRC>(a, s);
+    return signs ? launch_cols<BF16, FMT, SR, 32, true, DB, AMAX_ONLY, FP4SRC>(a, s)
+                 : launch_cols<BF16, FMT, SR, 32, false, DB, AMAX_ONLY, FP4SRC>(a, s);
 }
 
-template <bool BF16>
+template <bool BF16, bool FP4SRC = false>
 cudaError_t cols_by_fmt(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db, cudaStream_t s) {
-    if (fmt == MXFP4) return sr ? cols_by_rot<BF16, MXFP4, true, false, false>(a, rot_n, signs, s)
-                                : cols_by_rot<BF16, MXFP4, false, false, false>(a, rot_n, signs, s);
-    if (fmt == UFP4) return sr ? cols_by_rot<BF16, UFP4, true, false, false>(a, rot_n, signs, s)
-                               : cols_by_rot<BF16, UFP4, false, false, false>(a, rot_n, signs, s);
-    if (db) return sr ? cols_by_rot<BF16, NVFP4, true, true, false>(a, rot_n, signs, s)
-                      : cols_by_rot<BF16, NVFP4, false, true, false>(a, rot_n, signs, s);
-    return sr ? cols_by_rot<BF16, NVFP4, true, false, false>(a, rot_n, signs, s)
-              : cols_by_rot<BF16, NVFP4, false, false, false>(a, rot_n, signs, s);
+    if (fmt == MXFP4) return sr ? cols_by_rot<BF16, MXFP4, true, false, false, FP4SRC>(a, rot_n, signs, s)
+                                : cols_by_rot<BF16, MXFP4, false, false, false, FP4SRC>(a, rot_n, signs, s);
+    if (fmt == UFP4) return sr ? cols_by_rot<BF16, UFP4, true, false, false, FP4SRC>(a, rot_n, signs, s)
+                               : cols_by_rot<BF16, UFP4, false, false, false, FP4SRC>(a, rot_n, signs, s);
+    if (db) return sr ? cols_by_rot<BF16, NVFP4, true, true, false, FP4SRC>(a, rot_n, signs, s)
+                      : cols_by_rot<BF16, NVFP4, false, true, false, FP4SRC>(a, rot_n, signs, s);
+    return sr ? cols_by_rot<BF16, NVFP4, true, false, false, FP4SRC>(a, rot_n, signs, s)
+              : cols_by_rot<BF16, NVFP4, false, false, false, FP4SRC>(a, rot_n, signs, s);
 }
 
 }  // namespace
@@ -228,6 +278,15 @@ cudaError_t launch_quantize_cols(const QuantArgs& a, bool bf16, int fmt, bool sr
 cudaError_t launch_amax_cols(const QuantArgs& a, bool bf16, int rot_n, bool signs, cudaStream_t s) {
     return bf16 ? cols_by_rot<true, NVFP4, false, false, true>(a, rot_n, signs, s)
                 : cols_by_rot<false, NVFP4, false, false, true>(a, rot_n, signs, s);
+}
+
+cudaError_t launch_requantize_cols(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db,
+                                   cudaStream_t s) {
+    return cols_by_fmt<false, true>(a, fmt, sr, rot_n, signs, db, s);
+}
+
+cudaError_t launch_requant_amax_cols(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s) {
+    return cols_by_rot<false, NVFP4, false, false, true, true>(a, rot_n, signs, s);
 }
 
 }  // namespace fp4

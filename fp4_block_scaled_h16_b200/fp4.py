@@ -33,7 +33,7 @@ FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
 
 EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_quantize",
            "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit",
-           "fp4_quantize_noalloc")
+           "fp4_quantize_noalloc", "fp4_requantize")
 
 _P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_uint32, ctypes.c_size_t)
@@ -46,11 +46,14 @@ _lib.fp4_amax.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _P, _P]
 _lib.fp4_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _I, _U64, _U32, _P,
                               _P, _P, _P, _P, _P, _SZ, _P]
 _lib.fp4_quantize_noalloc.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P]
+_lib.fp4_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P, _P,
+                                _P, _SZ, _P]
 _lib.fp4_gemm.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P]
 _lib.fp4_last_error.argtypes = [_P]
 _lib.fp4_set_wait_limit.argtypes = [_U32]
 _lib.fp4_set_wait_limit.restype = None
-for _f in ("fp4_amax", "fp4_quantize", "fp4_quantize_noalloc", "fp4_gemm", "fp4_last_error", "fp4_quantize_workspace_size"):
+for _f in ("fp4_amax", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
+           "fp4_quantize_workspace_size"):
     getattr(_lib, _f).restype = _I
 
 
@@ -113,6 +116,33 @@ def fp4_quantize(x, in_dtype, rows, cols, ld, fmt, rounding, rotation, axis, dou
                              int(double_block), seed, tensor_id, _ptr(tensor_amax), _ptr(codes),
                              _ptr(scales), _ptr(outer_scales), _ptr(tensor_scale), _ptr(workspace),
                              workspace_bytes, _stream(stream)), "fp4_quantize")
+
+
+def fp4_requantize(src_codes, src_scales, src_outer, src_tensor_scale, lines, K, src_fmt, src_double_block,
+                   fmt, rounding, rotation, double_block, seed, tensor_id, tensor_amax, codes, scales,
+                   outer_scales, tensor_scale, workspace, workspace_bytes, stream=None) -> None:
+    _check(_lib.fp4_requantize(_ptr(src_codes), _ptr(src_scales), _ptr(src_outer), _ptr(src_tensor_scale),
+                               lines, K, src_fmt, int(src_double_block), fmt, rounding, rotation,
+                               int(double_block), seed, tensor_id, _ptr(tensor_amax), _ptr(codes), _ptr(scales),
+                               _ptr(outer_scales), _ptr(tensor_scale), _ptr(workspace), workspace_bytes,
+                               _stream(stream)), "fp4_requantize")
+
+
+def requantize(q, fmt, rounding=FP4_RTNE, rotation=FP4_ROT_NONE, double_block=False, seed=0, tensor_id=0,
+               tensor_amax=None, out=None, workspace=None, stream=None):
+    """Re-quantize the quantized tensor q (lines x K) along the other axis: the
+    result has K lines of q["lines"] elements (fp4_requantize)."""
+    import torch
+    lines, K = q["lines"], q["K"]
+    r = out if out is not None else alloc_qtensor(K, lines, fmt, double_block, q["codes"].device)
+    ws_bytes = fp4_quantize_workspace_size(fmt, double_block, tensor_amax is not None)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q["codes"].device)
+    fp4_requantize(q["codes"], q["scales"], q["outer"], q["tensor_scale"] if q["format"] != FP4_MXFP4 else None,
+                   lines, K, q["format"], q["double_block"], fmt, rounding, rotation, double_block, seed,
+                   tensor_id, tensor_amax, r["codes"], r["scales"], r["outer"], r["tensor_scale"],
+                   workspace if ws_bytes else None, ws_bytes, stream)
+    return r
 
 
 def fp4_quantize_noalloc(x, in_dtype, rows, cols, ld, fmt, rounding, rotation, axis, seed, tensor_id,

@@ -179,6 +179,43 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
                           void* stream);
 
 /*
+ * fp4_requantize -- re-quantize an already quantized tensor along the other
+ * axis.  "TetraJet-v2", section 2.A: the backward pass estimates with X^, the
+ * dequantized forward operand, rather than X ("aligning the tensors"), and the
+ * 1x16 weight groups need a matching alignment for the transposed weight.  The
+ * Dgrad / Wgrad operand is therefore the forward tensor's dequantized values
+ * quantized along the transposed axis, not the original bf16 tensor.
+ *
+ * The source is a quantized tensor of `lines` lines with K elements each,
+ * read as the logical matrix X^ [lines, K].  Each element of X^ is the
+ * dequantized value rounded once to binary32: RN(q * s_block * s_ref), with
+ * s_ref the tensor scale, the outer scale (double block) or 1 (MXFP4).  The
+ * product q * s_block is exact in binary32.  The result is what fp4_quantize
+ * gives for that binary32 X^ with axis = 0: K lines of `lines` elements, with
+ * the same rotation, scale, rounding and SR-counter rules (element (r, c) of
+ * X^ has index i = r * K + c).  The source must not be rotated: undoing a
+ * rotation along the source axis is not part of this call.
+ *
+ * Arguments
+ *   src_codes, src_scales, src_outer, src_tensor_scale, lines, K,
+ *   src_format, src_double_block   the source, laid out as fp4_quantize
+ *                                  writes it (src_outer for double block,
+ *                                  src_tensor_scale for NVFP4 / UFP4 without it)
+ *   format ... workspace_bytes     the result, as in fp4_quantize, for an
+ *                                  input of `lines` rows and K columns on axis 0
+ * Shape rules: K % 16 == 0 and K % (source block) == 0 (128 for a double-block
+ * source); `lines` % (result block) == 0, % rotation size, % 128 for a
+ * double-block result.  src_codes and codes 16-byte aligned.  Errors as
+ * fp4_quantize; nothing is launched on an error.
+ */
+fp4_status_t fp4_requantize(const uint8_t* src_codes, const uint8_t* src_scales, const float* src_outer,
+                            const float* src_tensor_scale, int64_t lines, int64_t K, fp4_format_t src_format,
+                            int src_double_block, fp4_format_t format, fp4_rounding_t rounding,
+                            fp4_rotation_t rotation, int double_block, uint64_t seed, uint32_t tensor_id,
+                            const float* tensor_amax, uint8_t* codes, uint8_t* scales, float* outer_scales,
+                            float* tensor_scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fp4_quantize_noalloc -- fp4_quantize for NVFP4 / UFP4 with the tensor scale
  * taken from an internal amax, for callers that cannot allocate device
  * memory: code running where cudaMalloc is unavailable or forbidden (a plug-in

@@ -271,6 +271,28 @@ def dequantize(q: dict) -> np.ndarray:
     return out
 
 
+def dequantize32(q: dict) -> np.ndarray:
+    """X^ in binary32: each exact dequantized value rounded once to nearest-even.
+
+    "TetraJet-v2" 2.A (aligning the tensors in the backward pass: estimating
+    with X^ rather than X).  The pages fix no precision for X^; the reading is
+    one rounding of the exact product q * s_block * s_ref."""
+    return dequantize(q).astype(np.float32)
+
+
+def requantize(q: dict, fmt: int, rounding: int = RTNE, rotation: int = ROT_NONE,
+               double_block: bool = False, seed: int = 0, tensor_id: int = 0,
+               amax: float | None = None, lines=None, threads: int | None = None) -> dict:
+    """Re-quantize the quantized tensor q ([n, K], lines along K) along the
+    transposed axis: X^ = dequantize32(q), read as an [n, K] row-major tensor,
+    quantized with axis 0 ("TetraJet-v2" 2.A: X^ for the backward pass, the
+    transposed weight's 1x16 groups re-aligned).  The result has K lines of n
+    elements; SR counters follow the [n, K] indexing of X^."""
+    return quantize(dequantize32(q), fmt, rounding=rounding, rotation=rotation, axis=0,
+                    double_block=double_block, seed=seed, tensor_id=tensor_id, amax=amax,
+                    lines=lines, threads=threads)
+
+
 def gemm(qa: dict, qb: dict):
     """C64 = deq(A) @ deq(B)^T in float64 and the bound sum_k |a_ik b_jk|.
 

@@ -104,6 +104,36 @@ def test_empty_gemm_is_a_no_op():
     assert g(M=0) == 0 and g(N=0, ldc=0) == 0
 
 
+def rq(**kw):
+    args = dict(sc=ADDR, ss=ADDR, so=None, sts=ADDR, lines=256, K=512, sfmt=fp4.FP4_NVFP4, sdb=0,
+                fmt=fp4.FP4_NVFP4, rounding=fp4.FP4_SR, rotation=fp4.FP4_ROT_NONE, db=0, seed=0, tid=0,
+                amax=None, codes=ADDR, scales=ADDR, outer=None, ts=ADDR, ws=ADDR, wsb=256)
+    args.update(kw)
+    a = args
+    return fp4._lib.fp4_requantize(a["sc"], a["ss"], a["so"], a["sts"], a["lines"], a["K"], a["sfmt"], a["sdb"],
+                                   a["fmt"], a["rounding"], a["rotation"], a["db"], a["seed"], a["tid"], a["amax"],
+                                   a["codes"], a["scales"], a["outer"], a["ts"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(sfmt=3), 1), (dict(fmt=5), 1), (dict(rounding=2), 1), (dict(rotation=7), 1), (dict(sdb=2), 1),
+    (dict(sdb=1, sfmt=fp4.FP4_MXFP4), 1), (dict(db=1, fmt=fp4.FP4_UFP4), 1), (dict(lines=-1), 1),
+    (dict(sc=None), 1), (dict(sts=None), 1), (dict(sdb=1, so=None), 1), (dict(codes=None), 1),
+    (dict(db=1, outer=None), 1), (dict(ts=None), 1),
+    (dict(K=520), 2), (dict(sfmt=fp4.FP4_MXFP4, K=528), 2), (dict(sdb=1, so=ADDR, K=576), 2),
+    (dict(lines=264), 2), (dict(fmt=fp4.FP4_MXFP4, lines=272), 2), (dict(rotation=fp4.FP4_ROT_H32, lines=272), 2),
+    (dict(db=1, outer=ADDR, lines=320), 2),
+    (dict(sc=ADDR + 8), 3), (dict(codes=ADDR + 4), 3), (dict(so=ADDR + 2, sdb=1), 3),
+    (dict(ws=None), 4), (dict(wsb=8), 4),
+])
+def test_requantize_host_validation(kw, status):
+    assert rq(**kw) == status
+
+
+def test_empty_requantize_is_a_no_op_without_gpu_work():
+    assert rq(lines=0, sc=None, ss=None, codes=None, scales=None, ws=None) in (0, fp4.FP4_ERR_NO_DEVICE)
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
 def test_valid_call_without_gpu_reports_no_device():
     assert q() == fp4.FP4_ERR_NO_DEVICE
