@@ -24,7 +24,7 @@ __device__ __forceinline__ float fp4_code_value(uint32_t n, bool ufp4) {
 
 // FP4SRC: the tile is the dequantized source X^ (fp4_requantize) instead of x
 template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY, bool FP4SRC = false>
-__global__ void __launch_bounds__(T0_THREADS)
+__global__ void __launch_bounds__(T0_THREADS, 4)
 quant_cols_kernel(const QuantArgs a) {
     __shared__ __align__(16) float tile[T0_ROWS][T0_COLS + 4];
     __shared__ float chunk_max[4][T0_COLS];
