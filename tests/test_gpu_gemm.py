@@ -50,6 +50,22 @@ def test_gemm_on_oracle_operands(fp4, fmt, out_bf16, shape):
     assert_within_gemm_bound(C.float().cpu().numpy(), C64, bound, out_bf16, what=str((fmt, shape, out_bf16)))
 
 
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("shape", [(5120, 1024, 256), (2560, 2048, 512)])
+def test_gemm_with_more_tiles_than_sms_on_oracle_operands(fp4, fmt, shape):
+    # more 128x256 tiles than SMs (160 tiles on 148 SMs: a second, nearly
+    # empty wave of persistent tiles); every element against the oracle
+    M, N, K = shape
+    a, b = rand(M, K, M + fmt), rand(N, K, N + 7 + fmt, 0.1)
+    qa = oracle_quantize(a, fmt=fmt)
+    qb = oracle_quantize(b, fmt=fmt)
+    C64, bound = oracle.gemm(qa, qb)
+    C = fp4.gemm(upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb), fp4.FP4_OUT_BF16)
+    torch.cuda.synchronize()
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    assert_within_gemm_bound(C.float().cpu().numpy(), C64, bound, True, what=str((fmt, shape)))
+
+
 def test_gemm_ldc_larger_than_n(fp4):
     a, b = rand(128, 512, 1), rand(256, 512, 2)
     qa, qb = oracle_quantize(a, fmt=NV), oracle_quantize(b, fmt=NV)
