@@ -2,6 +2,7 @@
 // the columns of the row-major input and the output lines are its columns, as
 // the Dgrad / Wgrad operands need ("TetraJet-v2" 2.A: 1x16 groups re-aligned
 // for the transposed weight).  Same arithmetic as the row-axis kernel.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -20,6 +21,14 @@ __device__ __forceinline__ float fp4_code_value(uint32_t n, bool ufp4) {
     const uint32_t m = n & 7u;
     const float mag = ufp4 ? (float)m : (float)((0xC8643210u >> (4u * m)) & 0xFu) * 0.5f;   // twice the level
     return (n & 8u) ? -mag : mag;
+}
+
+// two E2M1 codes (one byte, element 2j in the low nibble) -> their grid values
+// as binary16, element 2j in the low half
+__device__ __forceinline__ __half2 e2m1x2_to_h2(uint32_t byte) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(byte));
+    return *reinterpret_cast<__half2*>(&r);
 }
 
 // FP4SRC: the tile is the dequantized source X^ (fp4_requantize) instead of x
@@ -66,10 +75,23 @@ quant_cols_kernel(const QuantArgs a) {
                     E = e4m3_to_f32(sb);
                     s_ref = a.src_db ? __ldg(a.src_outer + gr * (C / 128) + gc / 128) : ts;
                 }
+                if (ufp4) {
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const uint32_t n = ((k < 8 ? cw.x : cw.y) >> (4 * (k & 7))) & 0xFu;
-                    x[k] = __fmul_rn(__fmul_rn(fp4_code_value(n, ufp4), E), s_ref);
+                    for (int k = 0; k < 16; ++k) {
+                        const uint32_t n = ((k < 8 ? cw.x : cw.y) >> (4 * (k & 7))) & 0xFu;
+                        x[k] = __fmul_rn(__fmul_rn(fp4_code_value(n, true), E), s_ref);
+                    }
+                } else {
+                    // E2M1: codes decoded two at a time; q * E is exact in binary16
+                    // (at most 6 significant bits, between 2^-10 and 2688)
+                    const __half2 E2 = __float2half2_rn(E);
+#pragma unroll
+                    for (int b = 0; b < 8; ++b) {
+                        const uint32_t byte = ((b < 4 ? cw.x : cw.y) >> (8 * (b & 3))) & 0xFFu;
+                        const float2 qe = __half22float2(__hmul2(e2m1x2_to_h2(byte), E2));
+                        x[2 * b] = __fmul_rn(qe.x, s_ref);
+                        x[2 * b + 1] = __fmul_rn(qe.y, s_ref);
+                    }
                 }
             } else {
 #pragma unroll
