@@ -173,21 +173,48 @@ def run_gpu(args, rank, world, device):
     torch.cuda.synchronize()
     assert fp4.fp4_last_error() == fp4.FP4_OK
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # optionally the step as one CUDA graph (its 3 kernels and 2 workspace
+    # memsets), captured on a side stream after the eager warm-up
+    graph = None
+    if args.graph:
+        side = torch.cuda.Stream(device)
+        side.wait_stream(torch.cuda.current_stream(device))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            w.step()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(graph, stream=side):
+                w.step()
+        torch.cuda.current_stream(device).wait_stream(side)
+        torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(device.index) as clocks:
         for i in range(args.steps):
             flush()                       # L2 flush, outside the timed events
-            w.step(evs[i])
+            evs[i][0].record()
+            if graph is not None:
+                graph.replay()
+            else:
+                w.step()
+            evs[i][1].record()
         torch.cuda.synchronize()
     barrier()
-    qx = [e[0].elapsed_time(e[1]) for e in evs]
-    qw = [e[1].elapsed_time(e[2]) for e in evs]
-    gm = [e[2].elapsed_time(e[3]) for e in evs]
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_ms = sum(step_ms)
     status = fp4.fp4_last_error()
+
+    # the step's kernels one by one (eager, events between them)
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(max(3, min(args.steps, 20)))]
+    for e in evk:
+        flush()
+        w.step(e)
+    torch.cuda.synchronize()
+    qx = [e[0].elapsed_time(e[1]) for e in evk]
+    qw = [e[1].elapsed_time(e[2]) for e in evk]
+    gm = [e[2].elapsed_time(e[3]) for e in evk]
 
     # the two passes as separate kernels (fp4_amax, then fp4_quantize given the
     # amax), timed on a second pass: each kernel against its own bytes
@@ -264,6 +291,7 @@ def run_gpu(args, rank, world, device):
                    "rotation": "H16", "rounding": "RTNE", "out": "bf16",
                    "value_is": "GEMM FLOP of the step / whole step time (quantize X and W, each with its tensor amax, + GEMM)",
                    "l2": "flushed between steps (256 MiB write, then 256 MiB read, outside the timed events)",
+                   "launch": "the step replayed as one CUDA graph" if args.graph else "eager launches",
                    "parallelism": "independent problem per GPU" if world > 1 else "single GPU"},
         "roofline": {"bound": "tensor", "kernel": "gemm_kernel (NVFP4, 128x256 tile)",
                      "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
@@ -489,6 +517,8 @@ def main():
     ap.add_argument("--impl", choices=["fp4", "reference"], default="fp4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel table")
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step replayed as one CUDA graph (measured equal to eager launches)")
     ap.add_argument("--configs", default=",".join(CONFIG_NAMES),
                     help="comma-separated workloads of the per-config table: " + ", ".join(CONFIG_NAMES))
     args = ap.parse_args()
