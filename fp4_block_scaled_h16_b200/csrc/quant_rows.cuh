@@ -2,13 +2,25 @@
 // templates; instantiated per input type in quantize.cu / quantize_rows_f32.cu.
 //
 // Persistent CTAs stream the input through a ring of shared-memory stages
-// filled by bulk asynchronous copies (cp.async.bulk, completion on an
+// filled by bulk asynchronous copies (cp.async.bulk, completion on a "full"
 // mbarrier), so the bytes in flight cost no registers: up to STAGES-1 stages
-// of 16 KB per CTA are loading while one is computed.  A stage holds whole
-// lines when a line fits (one copy per line) or one segment of a long line.
-// Thread t of the CTA computes unit t of the stage: U = 32 contiguous
-// elements (16 when the line length is only a multiple of 16).  Double-block
-// 128-chunks span 128/U adjacent lanes and are reduced with shuffles.
+// of 16 KB per CTA are loading while one is computed.  Each warp copies its
+// units out to registers at the start of a stage and releases the slot on an
+// "empty" mbarrier; thread 0 refills the previous stage's slot, so warps never
+// wait for one another.  A stage holds whole lines when a line fits (one copy
+// per line) or one segment of a long line.  Thread t of the CTA computes unit
+// t of the stage: U = 32 contiguous elements (16 when the line length is only
+// a multiple of 16).  Double-block 128-chunks span 128/U adjacent lanes and
+// are reduced with shuffles.
+//
+// Modes: quantize with a known tensor amax; the amax alone (fp4_amax); or
+// both in one cooperative launch (fp4_quantize with the internal amax): the
+// CTAs run their stages once for the amax, meet at a bounded grid barrier,
+// and run them again, in reverse order, to quantize -- the second read of
+// the tensor then comes mostly from L2.  Every CTA must be resident for the
+// barrier, which the cooperative launch guarantees; work that other streams
+// keep on the SMs for more than the barrier's poll budget (about 2^22 sleeps
+// of 32 ns) makes it report FP4_ERR_TIMEOUT rather than wait longer.
 #pragma once
 
 #include "quant_common.cuh"
