@@ -294,11 +294,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 template <int FMT, int BN, bool OUT_BF16>
 cudaError_t run(const GemmArgs& g, cudaStream_t s) {
     using G = Cfg<FMT, BN>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_kernel<FMT, BN, OUT_BF16>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM);
+    static PerDeviceOnce setup;
+    const cudaError_t attr_err = setup.run([](int) {
+        return cudaFuncSetAttribute(gemm_kernel<FMT, BN, OUT_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)G::SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap ta, tb;

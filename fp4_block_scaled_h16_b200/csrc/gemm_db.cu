@@ -356,11 +356,10 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
 template <bool OUT_BF16>
 cudaError_t run_db(const GemmArgs& g, cudaStream_t s) {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_db_kernel<OUT_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)SMEM);
+    static PerDeviceOnce setup;
+    const cudaError_t attr_err = setup.run([](int) {
+        return cudaFuncSetAttribute(gemm_db_kernel<OUT_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap ta, tb;

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <mutex>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -72,6 +73,28 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 cudaError_t launch_gemm_db(const GemmArgs& g, cudaStream_t s);
 // 2-D TMA map over packed codes [rows, K/2] bytes: box 128 bytes x box_rows, 128-byte swizzle
 bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K, int box_rows);
+
+// One-time setup per device (kernel attributes and occupancy are properties of
+// the kernel on one device): run() calls init once for the current device and
+// returns its cached status afterwards.
+constexpr int kOnceDevices = 64;
+struct PerDeviceOnce {
+    std::mutex mu;
+    bool done[kOnceDevices] = {};
+    cudaError_t status[kOnceDevices] = {};
+    template <class F>
+    cudaError_t run(F&& init, int* dev_out = nullptr) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kOnceDevices) return cudaErrorInvalidDevice;
+        if (dev_out) *dev_out = dev;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            status[dev] = init(dev);
+            done[dev] = true;
+        }
+        return status[dev];
+    }
+};
 
 // device state
 int num_sms();

@@ -329,15 +329,17 @@ cudaError_t launch_rows(const QuantArgs& a, cudaStream_t s) {
     constexpr int ES = BF16 ? 2 : 4;
     using Ring = RowRing<BF16, U, SR, MODE>;
     auto kernel = quant_rows_kernel<BF16, FMT, SR, ROT, SIGNS, DB, MODE, U>;
-    static bool attr_set = false;   // per instantiation
-    static int resident = 0;        // CTAs per SM the launch can keep resident
-    if (!attr_set) {
+    static PerDeviceOnce setup;                  // per instantiation and device
+    static int resident_on[kOnceDevices];        // CTAs per SM the launch can keep resident
+    int dev = 0;
+    const cudaError_t se = setup.run([&](int d) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Ring::SMEM);
-        if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, RQ_THREADS, Ring::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident_on[d], kernel, RQ_THREADS, Ring::SMEM);
+        return e;
+    }, &dev);
+    if (se != cudaSuccess) return se;
+    const int resident = resident_on[dev];
     // stage, line and element indices inside the kernel are 32-bit
     if (a.L >= ((int64_t)1 << 31) || a.K >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     RowStages st{};
