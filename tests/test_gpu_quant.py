@@ -212,3 +212,18 @@ def test_one_launch_amax_matches_two_launches(fp4, shape, fmt, rounding, rot):
     assert fp4.fp4_last_error() == fp4.FP4_OK
     for key in ("codes", "scales", "tensor_scale"):
         assert torch.equal(one[key].view(torch.uint8), two[key].view(torch.uint8)), key
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("fmt,rounding,rot", [(NV, 0, 1), (UF, 1, 2), (NV, 1, 0)])
+def test_one_launch_strided_input_matches_oracle(fp4, dtype, fmt, rounding, rot):
+    # the one-launch (internal amax) row path on a view whose row pitch is
+    # wider than its rows, in both input types, against the oracle
+    R, C, ld = 300, 384, 448
+    full = make_input(R, ld, dtype, seed=R + ld + fmt)
+    x = full[:, :C]
+    kw = dict(fmt=fmt, rounding=rounding, rotation=rot, axis=1, seed=4, tensor_id=6)
+    g = gpu_quantize(fp4, full.cuda()[:, :C], cols=C, **kw)
+    o = oracle_quantize(x.contiguous(), **kw)
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    assert_quant_equal(g, o, what="strided one-launch " + str(kw))
