@@ -513,13 +513,16 @@ def cpu_baseline(d, target_s=10.0):
 def run_reference(args):
     """The oracle, as it stands, timed on the host cores on a bounded sample."""
     d = workloads.nvfp4_fprop_qkv(seed=0)
-    budget_s = 120.0
-    rows = 64
-    t_cal, cores = oracle_slab_time(d, rows)
-    per_step_real = t_cal * rows / M + t_cal * rows * rows / (M * N)   # rough real seconds per slab step
+    budget_s = 120.0                              # wall time of the whole run
     steps = args.steps + args.warmup
-    if per_step_real * steps > budget_s:
-        rows = 16
+    # calibrate on a 64-row slab, then take the largest slab (a multiple of 16
+    # rows, at most 1024) whose steps fit the budget: small slabs are
+    # dominated by fixed costs and understate the oracle's rate
+    t0 = time.perf_counter()
+    oracle_slab_time(d, 64)
+    wall64 = time.perf_counter() - t0
+    rows = int(64 * budget_s / (steps * max(wall64, 1e-4)))
+    rows = max(16, min(1024, rows - rows % 16))
     times = []
     for i in range(args.warmup + args.steps):
         t, cores = oracle_slab_time(d, rows)
