@@ -72,6 +72,9 @@ struct GemmParams {
     int M, N, K;
     int nb4;          // scale atoms per 128 rows along K
     int tiles_m, tiles_n;
+    // work units: tiles [0, split_base) whole; the tiles after it (a last wave
+    // that would fill at most half the SMs) as two halves of BN / 2 columns
+    int units, split_base;
     uint32_t wait_limit;
     unsigned int* err;
 };
@@ -81,10 +84,59 @@ __device__ __forceinline__ void raise_timeout(const GemmParams& p, volatile int*
     atomicExch(p.err, ERR_TIMEOUT);
 }
 
+// output block of work unit u: rows m0.., columns n0.. (BN of them, or BN / 2
+// for a half unit)
+template <int BN>
+__device__ __forceinline__ bool unit_geom(const GemmParams& p, int u, int& m0, int& n0) {
+    if (u < p.split_base) {
+        m0 = (u % p.tiles_m) * BM;
+        n0 = (u / p.tiles_m) * BN;
+        return false;
+    }
+    const int t = p.split_base + ((u - p.split_base) >> 1);
+    m0 = (t % p.tiles_m) * BM;
+    n0 = (t / p.tiles_m) * BN + ((u - p.split_base) & 1) * (BN / 2);
+    return true;
+}
+
+// one stage's scale-factor copies and MMAs into the accumulator at `tmem`,
+// NMMA columns wide (BN, or BN / 2 for a half unit)
+template <int FMT, int BN, int NMMA>
+__device__ __forceinline__ void mma_stage(uint32_t tmem, uint32_t st, int kt) {
+    using G = Cfg<FMT, BN>;
+    const uint32_t st_sfa = st + G::A_BYTES + G::B_BYTES;
+    const uint32_t st_sfb = st_sfa + G::SFA_BYTES;
+#pragma unroll
+    for (int j = 0; j < G::ATOMS; ++j) {
+        sm100::tc_cp_sf(tmem + G::SFA_COL + 4 * j, sm100::desc_sf(st_sfa + 512 * j));
+#pragma unroll
+        for (int rb = 0; rb < NMMA / 128; ++rb)
+            sm100::tc_cp_sf(tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * j + 4 * rb,
+                            sm100::desc_sf(st_sfb + (rb * G::ATOMS + j) * 512));
+    }
+#pragma unroll
+    for (int kk = 0; kk < BK / 64; ++kk) {
+        const uint64_t da = sm100::desc_sw128(st + 32 * kk);
+        const uint64_t db = sm100::desc_sw128(st + G::A_BYTES + 32 * kk);
+        const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
+        if (FMT == MXFP4) {
+            // block 32: two scale bytes per MMA, the pair kk % 2 of atom kk / 2
+            const int j = kk / 2;
+            const uint32_t id = sm100::idesc_block_scaled(NMMA, true, (kk & 1) * 2, (kk & 1) * 2);
+            sm100::mma_mxf4(tmem, da, db, id, tmem + G::SFA_COL + 4 * j,
+                            tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * j, acc);
+        } else {
+            const uint32_t id = sm100::idesc_block_scaled(NMMA, false, 0, 0);
+            sm100::mma_nvf4(tmem, da, db, id, tmem + G::SFA_COL + 4 * kk,
+                            tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * kk, acc);
+        }
+    }
+}
+
 template <int FMT, int BN, bool OUT_BF16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const GemmParams p) {
+            const __grid_constant__ CUtensorMap tmBh, const GemmParams p) {
     using G = Cfg<FMT, BN>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base (the 128-byte swizzle atoms need it)
@@ -111,6 +163,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         sm100::fence_barrier_init();
         sm100::prefetch_tmap(&tmA);
         sm100::prefetch_tmap(&tmB);
+        if (p.units > p.split_base) sm100::prefetch_tmap(&tmBh);
     }
     if (warp == 1) {
         sm100::tmem_alloc(tmem_slot, TMEM_COLS);
@@ -121,7 +174,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    const int tiles = p.tiles_m * p.tiles_n;
     const int kt_count = p.K / BK;
 
     if (warp == 0) {
@@ -131,8 +183,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             uint32_t phase = 0;
             uint32_t fills = 0;           // fill i went to stage i % STAGES, phase i / STAGES
             bool ok = true;
-            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN;
+            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+                int m0, n0;
+                const bool half_unit = unit_geom<BN>(p, u, m0, n0);
                 for (int kt = 0; kt < kt_count; ++kt) {
                     if (!sm100::mbar_wait(&empty[stage], phase ^ 1u, p.wait_limit, abort_flag)) {
                         raise_timeout(p, abort_flag);
@@ -140,17 +193,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                         break;
                     }
                     uint8_t* st = smem + stage * G::STAGE_BYTES;
-                    sm100::mbar_arrive_expect_tx(&full[stage], G::TX);
-                    sm100::tma_load_2d(st, &tmA, kt * (BK / 2), m0, &full[stage]);
-                    sm100::tma_load_2d(st + G::A_BYTES, &tmB, kt * (BK / 2), n0, &full[stage]);
                     const int kb0 = kt * G::KB;                          // first scale column
                     const uint8_t* sfa = p.a_sf + ((int64_t)(m0 / 128) * p.nb4 + kb0 / 4) * 512;
-                    sm100::bulk_load(st + G::A_BYTES + G::B_BYTES, sfa, G::SFA_BYTES, &full[stage]);
+                    if (BN == 256 && half_unit) {
+                        // 128 columns: half of B and of its scales
+                        sm100::mbar_arrive_expect_tx(&full[stage], G::A_BYTES + G::SFA_BYTES + G::B_BYTES / 2 +
+                                                                       G::ATOMS * 512);
+                        sm100::tma_load_2d(st, &tmA, kt * (BK / 2), m0, &full[stage]);
+                        sm100::tma_load_2d(st + G::A_BYTES, &tmBh, kt * (BK / 2), n0, &full[stage]);
+                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES, sfa, G::SFA_BYTES, &full[stage]);
+                        const uint8_t* sfb = p.b_sf + ((int64_t)(n0 / 128) * p.nb4 + kb0 / 4) * 512;
+                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES, sfb, G::ATOMS * 512,
+                                         &full[stage]);
+                    } else {
+                        sm100::mbar_arrive_expect_tx(&full[stage], G::TX);
+                        sm100::tma_load_2d(st, &tmA, kt * (BK / 2), m0, &full[stage]);
+                        sm100::tma_load_2d(st + G::A_BYTES, &tmB, kt * (BK / 2), n0, &full[stage]);
+                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES, sfa, G::SFA_BYTES, &full[stage]);
 #pragma unroll
-                    for (int rb = 0; rb < BN / 128; ++rb) {
-                        const uint8_t* sfb = p.b_sf + ((int64_t)(n0 / 128 + rb) * p.nb4 + kb0 / 4) * 512;
-                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES + rb * G::ATOMS * 512,
-                                         sfb, G::ATOMS * 512, &full[stage]);
+                        for (int rb = 0; rb < BN / 128; ++rb) {
+                            const uint8_t* sfb = p.b_sf + ((int64_t)(n0 / 128 + rb) * p.nb4 + kb0 / 4) * 512;
+                            sm100::bulk_load(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES + rb * G::ATOMS * 512,
+                                             sfb, G::ATOMS * 512, &full[stage]);
+                        }
                     }
                     ++fills;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -170,7 +235,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, issued = false;
-            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+                const bool half_unit = u >= p.split_base;
                 if (!sm100::mbar_wait(acc_empty, acc_phase ^ 1u, p.wait_limit, abort_flag)) {
                     raise_timeout(p, abort_flag);
                     break;
@@ -184,33 +250,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     }
                     sm100::tc_fence_after();
                     const uint32_t st = sm100::smem_u32(smem + stage * G::STAGE_BYTES);
-                    const uint32_t st_sfa = st + G::A_BYTES + G::B_BYTES;
-                    const uint32_t st_sfb = st_sfa + G::SFA_BYTES;
-#pragma unroll
-                    for (int j = 0; j < G::ATOMS; ++j) {
-                        sm100::tc_cp_sf(tmem + G::SFA_COL + 4 * j, sm100::desc_sf(st_sfa + 512 * j));
-#pragma unroll
-                        for (int rb = 0; rb < BN / 128; ++rb)
-                            sm100::tc_cp_sf(tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * j + 4 * rb,
-                                            sm100::desc_sf(st_sfb + (rb * G::ATOMS + j) * 512));
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < BK / 64; ++kk) {
-                        const uint64_t da = sm100::desc_sw128(st + 32 * kk);
-                        const uint64_t db = sm100::desc_sw128(st + G::A_BYTES + 32 * kk);
-                        const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
-                        if (FMT == MXFP4) {
-                            // block 32: two scale bytes per MMA, the pair kk % 2 of atom kk / 2
-                            const int j = kk / 2;
-                            const uint32_t id = sm100::idesc_block_scaled(BN, true, (kk & 1) * 2, (kk & 1) * 2);
-                            sm100::mma_mxf4(tmem, da, db, id, tmem + G::SFA_COL + 4 * j,
-                                            tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * j, acc);
-                        } else {
-                            const uint32_t id = sm100::idesc_block_scaled(BN, false, 0, 0);
-                            sm100::mma_nvf4(tmem, da, db, id, tmem + G::SFA_COL + 4 * kk,
-                                            tmem + G::SFB_COL + G::SFB_COLS_PER_ATOM * kk, acc);
-                        }
-                    }
+                    if (BN == 256 && half_unit) mma_stage<FMT, BN, (BN == 256 ? 128 : BN)>(tmem, st, kt);
+                    else mma_stage<FMT, BN, BN>(tmem, st, kt);
                     issued = true;
                     sm100::tc_commit(&empty[stage]);          // stage free once these MMAs are done
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -233,8 +274,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         float alpha = 1.0f;
         if (FMT == NVFP4) alpha = __fmul_rn(*p.a_ts, *p.b_ts);
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN + half * COLS;
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+            int m0, n0;
+            const bool half_unit = unit_geom<BN>(p, u, m0, n0);
+            n0 += half * COLS;
+            // a half unit has BN / 2 columns: the second column half's warps only hand over
+            const bool idle = half_unit && half == 1;
             // one lane polls, the warp follows its verdict (the TMEM loads below
             // are warp-collective)
             int got = 0;
@@ -243,6 +288,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 if (!got) raise_timeout(p, abort_flag);
             }
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
+            if (idle) {
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(acc_empty);
+                acc_phase ^= 1u;
+                continue;
+            }
             sm100::tc_fence_after();
             uint32_t r[COLS];
 #pragma unroll
@@ -300,8 +351,9 @@ cudaError_t run(const GemmArgs& g, cudaStream_t s) {
                                     (int)G::SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    CUtensorMap ta, tb;
-    if (!make_codes_map(&ta, g.a_codes, g.M, g.K, BM) || !make_codes_map(&tb, g.b_codes, g.N, g.K, BN))
+    CUtensorMap ta, tb, tbh;
+    if (!make_codes_map(&ta, g.a_codes, g.M, g.K, BM) || !make_codes_map(&tb, g.b_codes, g.N, g.K, BN) ||
+        !make_codes_map(&tbh, g.b_codes, g.N, g.K, BN / 2))
         return cudaErrorInvalidValue;
     GemmParams p{};
     p.a_sf = g.a_scales;
@@ -320,7 +372,13 @@ cudaError_t run(const GemmArgs& g, cudaStream_t s) {
     p.err = device_error_word();
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    gemm_kernel<FMT, BN, OUT_BF16><<<grid, NUM_THREADS, G::SMEM, s>>>(ta, tb, p);
+    // a last wave that would leave more than half the SMs idle runs as half
+    // tiles (BN = 256 only), so the tail takes about half as long
+    const int full_waves = tiles / grid, tail = tiles - full_waves * grid;
+    const bool split = BN == 256 && full_waves > 0 && tail > 0 && 2 * tail <= grid;
+    p.split_base = split ? full_waves * grid : tiles;
+    p.units = split ? p.split_base + 2 * tail : tiles;
+    gemm_kernel<FMT, BN, OUT_BF16><<<grid, NUM_THREADS, G::SMEM, s>>>(ta, tb, tbh, p);
     return cudaGetLastError();
 }
 
