@@ -37,10 +37,10 @@ WORKLOAD = "nvfp4_fprop_qkv_%dx%dx%d" % (M, N, K)
 GEMM_FLOP = 2.0 * M * N * K
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gemm_kernel
-# launch on this workload, from one ncu capture of the current kernel: 36.4 MB
-# read (the 33 MB of operands cross DRAM once) and 49.7 MB written (the rest of
+# launch on this workload, from one ncu capture of the current kernel: 36.3 MB
+# read (the 33 MB of operands cross DRAM once) and 50.6 MB written (the rest of
 # the 100.7 MB of C was still in L2 when the kernel ended)
-GEMM_TRAFFIC_BYTES = 36_395_520 + 49_682_944
+GEMM_TRAFFIC_BYTES = 36_305_152 + 50_610_176
 
 
 class L2Flush:
