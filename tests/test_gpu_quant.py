@@ -227,3 +227,20 @@ def test_one_launch_strided_input_matches_oracle(fp4, dtype, fmt, rounding, rot)
     o = oracle_quantize(x.contiguous(), **kw)
     assert fp4.fp4_last_error() == fp4.FP4_OK
     assert_quant_equal(g, o, what="strided one-launch " + str(kw))
+
+
+# Row lines whose length is an odd multiple of 16 run the row kernel with one
+# 16-element unit per thread (the tensor-scaled formats without a 32-rotation);
+# the shapes give many lines per stage with a ragged last stage, and lines
+# longer than one stage (split into segments, the last one ragged).
+@pytest.mark.parametrize("shape", [(300, 272, 280), (7, 48, 48), (5, 4112, 4112)])
+@pytest.mark.parametrize("fmt,rounding,rot", [(NV, 0, 0), (NV, 0, 1), (NV, 1, 3), (UF, 0, 1), (UF, 1, 0)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_row_lines_of_odd_sixteens(fp4, shape, fmt, rounding, rot, dtype):
+    R, C, ld = shape
+    x = make_input(R, ld, dtype, seed=R + C + 10 * fmt + rot, outliers=R >= 2)
+    kw = dict(fmt=fmt, rounding=rounding, rotation=rot, axis=1, seed=21, tensor_id=5)
+    g = gpu_quantize(fp4, x.cuda(), cols=C, **kw)
+    o = oracle_quantize(x, cols=C, **kw)
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    assert_quant_equal(g, o, what="odd-16 lines %s %s" % (shape, kw))
