@@ -38,9 +38,9 @@ GEMM_FLOP = 2.0 * M * N * K
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gemm_kernel
 # launch on this workload, from one ncu capture of the current kernel: 36.3 MB
-# read (the 33 MB of operands cross DRAM once) and 50.6 MB written (the rest of
+# read (the 33 MB of operands cross DRAM once) and 49.5 MB written (the rest of
 # the 100.7 MB of C was still in L2 when the kernel ended)
-GEMM_TRAFFIC_BYTES = 36_305_152 + 50_610_176
+GEMM_TRAFFIC_BYTES = 36_268_032 + 49_481_728
 
 
 class L2Flush:

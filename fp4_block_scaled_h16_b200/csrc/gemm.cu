@@ -100,14 +100,19 @@ __device__ __forceinline__ bool unit_geom(const GemmParams& p, int u, int& m0, i
 }
 
 // one stage's scale-factor copies and MMAs into the accumulator at `tmem`,
-// NMMA columns wide (BN, or BN / 2 for a half unit)
+// NMMA columns wide (BN, or BN / 2 for a half unit); a half-K stage (the last
+// one when K is an odd multiple of 128) holds the first BK / 2 elements of K
+// only: half the scale atoms, and the MMAs over its first two 64-K slices
 template <int FMT, int BN, int NMMA>
-__device__ __forceinline__ void mma_stage(uint32_t tmem, uint32_t st, int kt) {
+__device__ __forceinline__ void mma_stage(uint32_t tmem, uint32_t st, int kt, bool half_k) {
     using G = Cfg<FMT, BN>;
     const uint32_t st_sfa = st + G::A_BYTES + G::B_BYTES;
     const uint32_t st_sfb = st_sfa + G::SFA_BYTES;
+    const int atoms = half_k ? G::ATOMS / 2 : G::ATOMS;
+    const int slices = half_k ? BK / 128 : BK / 64;
 #pragma unroll
     for (int j = 0; j < G::ATOMS; ++j) {
+        if (j >= atoms) break;
         sm100::tc_cp_sf(tmem + G::SFA_COL + 4 * j, sm100::desc_sf(st_sfa + 512 * j));
 #pragma unroll
         for (int rb = 0; rb < NMMA / 128; ++rb)
@@ -116,6 +121,7 @@ __device__ __forceinline__ void mma_stage(uint32_t tmem, uint32_t st, int kt) {
     }
 #pragma unroll
     for (int kk = 0; kk < BK / 64; ++kk) {
+        if (kk >= slices) break;
         const uint64_t da = sm100::desc_sw128(st + 32 * kk);
         const uint64_t db = sm100::desc_sw128(st + G::A_BYTES + 32 * kk);
         const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
@@ -174,7 +180,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    const int kt_count = p.K / BK;
+    // stages per unit; with K an odd multiple of 128 the last one is half a
+    // stage: its code boxes reach past K (the tensor maps fill zeros there)
+    // and it carries half the scale atoms
+    const int kt_count = (p.K + BK - 1) / BK;
+    const bool ragged_k = (p.K % BK) != 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -195,26 +205,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     uint8_t* st = smem + stage * G::STAGE_BYTES;
                     const int kb0 = kt * G::KB;                          // first scale column
                     const uint8_t* sfa = p.a_sf + ((int64_t)(m0 / 128) * p.nb4 + kb0 / 4) * 512;
+                    // scale bytes per 128 rows in this stage (half of them in a half-K stage;
+                    // the code boxes always count whole, zero-filled past K)
+                    const uint32_t sf = (ragged_k && kt == kt_count - 1) ? G::ATOMS * 256 : G::ATOMS * 512;
                     if (BN == 256 && half_unit) {
                         // 128 columns: half of B and of its scales
-                        sm100::mbar_arrive_expect_tx(&full[stage], G::A_BYTES + G::SFA_BYTES + G::B_BYTES / 2 +
-                                                                       G::ATOMS * 512);
+                        sm100::mbar_arrive_expect_tx(&full[stage], G::A_BYTES + G::B_BYTES / 2 + 2 * sf);
                         sm100::tma_load_2d(st, &tmA, kt * (BK / 2), m0, &full[stage]);
                         sm100::tma_load_2d(st + G::A_BYTES, &tmBh, kt * (BK / 2), n0, &full[stage]);
-                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES, sfa, G::SFA_BYTES, &full[stage]);
+                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES, sfa, sf, &full[stage]);
                         const uint8_t* sfb = p.b_sf + ((int64_t)(n0 / 128) * p.nb4 + kb0 / 4) * 512;
-                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES, sfb, G::ATOMS * 512,
-                                         &full[stage]);
+                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES, sfb, sf, &full[stage]);
                     } else {
-                        sm100::mbar_arrive_expect_tx(&full[stage], G::TX);
+                        sm100::mbar_arrive_expect_tx(&full[stage], G::A_BYTES + G::B_BYTES + (1 + BN / 128) * sf);
                         sm100::tma_load_2d(st, &tmA, kt * (BK / 2), m0, &full[stage]);
                         sm100::tma_load_2d(st + G::A_BYTES, &tmB, kt * (BK / 2), n0, &full[stage]);
-                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES, sfa, G::SFA_BYTES, &full[stage]);
+                        sm100::bulk_load(st + G::A_BYTES + G::B_BYTES, sfa, sf, &full[stage]);
 #pragma unroll
                         for (int rb = 0; rb < BN / 128; ++rb) {
                             const uint8_t* sfb = p.b_sf + ((int64_t)(n0 / 128 + rb) * p.nb4 + kb0 / 4) * 512;
                             sm100::bulk_load(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES + rb * G::ATOMS * 512,
-                                             sfb, G::ATOMS * 512, &full[stage]);
+                                             sfb, sf, &full[stage]);
                         }
                     }
                     ++fills;
@@ -250,8 +261,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     }
                     sm100::tc_fence_after();
                     const uint32_t st = sm100::smem_u32(smem + stage * G::STAGE_BYTES);
-                    if (BN == 256 && half_unit) mma_stage<FMT, BN, (BN == 256 ? 128 : BN)>(tmem, st, kt);
-                    else mma_stage<FMT, BN, BN>(tmem, st, kt);
+                    const bool half_k = ragged_k && kt == kt_count - 1;
+                    if (BN == 256 && half_unit) mma_stage<FMT, BN, (BN == 256 ? 128 : BN)>(tmem, st, kt, half_k);
+                    else mma_stage<FMT, BN, BN>(tmem, st, kt, half_k);
                     issued = true;
                     sm100::tc_commit(&empty[stage]);          // stage free once these MMAs are done
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }

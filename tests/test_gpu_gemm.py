@@ -36,7 +36,8 @@ def rand(M, K, seed, scale=1.0):
 
 @pytest.mark.parametrize("out_bf16", [False, True])
 @pytest.mark.parametrize("fmt", [MX, NV])
-@pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 512), (384, 256, 1024), (128, 512, 2304)])
+@pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 512), (384, 256, 1024), (128, 512, 2304),
+                                   (128, 256, 128), (256, 128, 384), (384, 512, 1152)])
 def test_gemm_on_oracle_operands(fp4, fmt, out_bf16, shape):
     M, N, K = shape
     a, b = rand(M, K, M + K + fmt), rand(N, K, N + 3 * K + fmt, 0.1)
@@ -51,10 +52,11 @@ def test_gemm_on_oracle_operands(fp4, fmt, out_bf16, shape):
 
 
 @pytest.mark.parametrize("fmt", [MX, NV])
-@pytest.mark.parametrize("shape", [(5120, 1024, 256), (2560, 2048, 512)])
+@pytest.mark.parametrize("shape", [(5120, 1024, 256), (2560, 2048, 512), (5120, 1024, 384)])
 def test_gemm_with_more_tiles_than_sms_on_oracle_operands(fp4, fmt, shape):
     # more 128x256 tiles than SMs (160 tiles on 148 SMs: a second, nearly
-    # empty wave of persistent tiles); every element against the oracle
+    # empty wave of persistent tiles, run as 128-column halves; K = 384 ends
+    # on a half stage); every element against the oracle
     M, N, K = shape
     a, b = rand(M, K, M + fmt), rand(N, K, N + 7 + fmt, 0.1)
     qa = oracle_quantize(a, fmt=fmt)
