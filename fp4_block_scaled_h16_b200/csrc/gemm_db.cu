@@ -71,7 +71,10 @@ __device__ __forceinline__ void raise_timeout(const DbParams& p, volatile int* a
     atomicExch(p.err, ERR_TIMEOUT);
 }
 
-template <bool OUT_BF16>
+// PAIRED: K / 128 is even, and the promotion warps read the row outer scales
+// two chunks at a time (8-byte loads, half the load instructions); otherwise
+// one chunk at a time
+template <bool OUT_BF16, bool PAIRED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const DbParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -118,7 +121,10 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
 
     const int tiles = p.tiles_m * p.tiles_n;
-    const int kt_count = p.K / BK;
+    // stages per tile; with K an odd multiple of 128 the last stage holds one
+    // 128-K chunk (its code boxes read zeros past K, half its scale bytes)
+    const int kt_count = (p.K + BK - 1) / BK;
+    const bool ragged_k = (p.K % BK) != 0;
     const int nkc = p.K / 128;
 
     if (warp == 0) {
@@ -136,14 +142,16 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         break;
                     }
                     uint8_t* st = smem + stage * STAGE_BYTES;
-                    sm100::mbar_arrive_expect_tx(&full[stage], TX);
+                    const bool half_k = ragged_k && kt == kt_count - 1;
+                    const uint32_t sfa = half_k ? SFA_BYTES / 2 : SFA_BYTES, sfb = half_k ? SFB_BYTES / 2 : SFB_BYTES;
+                    sm100::mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES + sfa + sfb);
                     sm100::tma_load_2d(st, &tmA, kt * (BK / 2), m0, &full[stage]);
                     sm100::tma_load_2d(st + A_BYTES, &tmB, kt * (BK / 2), n0, &full[stage]);
                     const int kb0 = kt * (BK / 16);
                     sm100::bulk_load(st + A_BYTES + B_BYTES,
-                                     p.a_sf + ((int64_t)(m0 / 128) * p.nb4 + kb0 / 4) * 512, SFA_BYTES, &full[stage]);
+                                     p.a_sf + ((int64_t)(m0 / 128) * p.nb4 + kb0 / 4) * 512, sfa, &full[stage]);
                     sm100::bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES,
-                                     p.b_sf + ((int64_t)(n0 / 128) * p.nb4 + kb0 / 4) * 512, SFB_BYTES, &full[stage]);
+                                     p.b_sf + ((int64_t)(n0 / 128) * p.nb4 + kb0 / 4) * 512, sfb, &full[stage]);
                     ++fills;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -171,14 +179,18 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     sm100::tc_fence_after();
                     const uint32_t st = sm100::smem_u32(smem + stage * STAGE_BYTES);
                     const uint32_t st_sfa = st + A_BYTES + B_BYTES, st_sfb = st_sfa + SFA_BYTES;
+                    const int chunks = (ragged_k && kt == kt_count - 1) ? 1 : 2;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
+                        if (j >= 2 * chunks) break;
                         sm100::tc_cp_sf(tmem + SFA_COL + 4 * j, sm100::desc_sf(st_sfa + 512 * j));
                         sm100::tc_cp_sf(tmem + SFB_COL + 4 * j, sm100::desc_sf(st_sfb + 512 * j));
                     }
-                    // two 128-K chunks per stage, each into its own partial buffer
+                    // two 128-K chunks per stage (one in a half stage), each into its own
+                    // partial buffer
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
+                        if (h >= chunks) break;
                         if (!sm100::mbar_wait(&pempty[pb], ((pphase >> pb) & 1u) ^ 1u, p.wait_limit, abort_flag)) {
                             raise_timeout(p, abort_flag);
                             ok = false;
@@ -252,10 +264,20 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             float2 acc[COLS / 2];
 #pragma unroll
             for (int c = 0; c < COLS / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
-            // row outer scales two chunks at a time (K / 128 is even), one pair ahead
-            const float2* a_outer_row = reinterpret_cast<const float2*>(p.a_outer + (int64_t)row * nkc);
-            float2 sa_cur = __ldg(a_outer_row);
-            float2 sa_nxt = nkc > 2 ? __ldg(a_outer_row + 1) : sa_cur;
+            // the row's outer scales, loaded ahead of their use: in pairs (PAIRED,
+            // one pair ahead) or one at a time (three chunks ahead)
+            const float* a_outer_row = p.a_outer + (int64_t)row * nkc;
+            const float2* a_outer_pairs = reinterpret_cast<const float2*>(a_outer_row);
+            float2 sa_cur = make_float2(0.0f, 0.0f), sa_nxt = make_float2(0.0f, 0.0f);
+            float sa0 = 0.0f, sa1 = 0.0f, sa2n = 0.0f;
+            if (PAIRED) {
+                sa_cur = __ldg(a_outer_pairs);
+                sa_nxt = nkc > 2 ? __ldg(a_outer_pairs + 1) : sa_cur;
+            } else {
+                sa0 = __ldg(a_outer_row);
+                sa1 = nkc > 1 ? __ldg(a_outer_row + 1) : 0.0f;
+                sa2n = nkc > 2 ? __ldg(a_outer_row + 2) : 0.0f;
+            }
             // the slice is read in two halves of 16 columns: one half's TMEM load
             // is in flight while the other half is promoted
             const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + cg * COLS;
@@ -269,7 +291,7 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 sm100::tmem_ld_wait_on(ra);
             }
             for (int kc = 0; kc < nkc && ok; ++kc) {
-                const float sa = (kc & 1) ? sa_cur.y : sa_cur.x;
+                const float sa = PAIRED ? ((kc & 1) ? sa_cur.y : sa_cur.x) : sa0;
                 const float2 sa2 = make_float2(sa, sa);
                 const float4* sb = reinterpret_cast<const float4*>(outer_tile + kc * BN);
                 sm100::tmem_ld16(tbase + BN * pb + HALF, rb);
@@ -290,9 +312,15 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 if (lane == 0) sm100::mbar_arrive(&pempty[pb]);     // the tensor core may refill it
                 pphase ^= 1u << pb;
                 pb = (pb + 1 == PBUF) ? 0 : pb + 1;
-                if (kc & 1) {
-                    sa_cur = sa_nxt;
-                    if (kc + 3 < nkc) sa_nxt = __ldg(a_outer_row + (kc + 3) / 2);
+                if (PAIRED) {
+                    if (kc & 1) {
+                        sa_cur = sa_nxt;
+                        if (kc + 3 < nkc) sa_nxt = __ldg(a_outer_pairs + (kc + 3) / 2);
+                    }
+                } else {
+                    sa0 = sa1;
+                    sa1 = sa2n;
+                    if (kc + 3 < nkc) sa2n = __ldg(a_outer_row + kc + 3);
                 }
                 bool next = false;
                 if (kc + 1 < nkc) {
@@ -354,11 +382,11 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
-template <bool OUT_BF16>
+template <bool OUT_BF16, bool PAIRED>
 cudaError_t run_db(const GemmArgs& g, cudaStream_t s) {
     static PerDeviceOnce setup;
     const cudaError_t attr_err = setup.run([](int) {
-        return cudaFuncSetAttribute(gemm_db_kernel<OUT_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        return cudaFuncSetAttribute(gemm_db_kernel<OUT_BF16, PAIRED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -382,7 +410,7 @@ cudaError_t run_db(const GemmArgs& g, cudaStream_t s) {
     p.err = device_error_word();
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    gemm_db_kernel<OUT_BF16><<<grid, NUM_THREADS, SMEM, s>>>(ta, tb, p);
+    gemm_db_kernel<OUT_BF16, PAIRED><<<grid, NUM_THREADS, SMEM, s>>>(ta, tb, p);
     return cudaGetLastError();
 }
 
@@ -390,7 +418,8 @@ cudaError_t run_db(const GemmArgs& g, cudaStream_t s) {
 
 cudaError_t launch_gemm_db(const GemmArgs& g, cudaStream_t s) {
     if (g.K / 128 > MAX_CHUNKS) return cudaErrorInvalidValue;
-    return g.out_bf16 ? run_db<true>(g, s) : run_db<false>(g, s);
+    if ((g.K / 128) % 2 == 0) return g.out_bf16 ? run_db<true, true>(g, s) : run_db<false, true>(g, s);
+    return g.out_bf16 ? run_db<true, false>(g, s) : run_db<false, false>(g, s);
 }
 
 }  // namespace fp4

@@ -263,8 +263,8 @@ fp4_status_t fp4_quantize_noalloc(const void* x, fp4_in_dtype_t in_dtype, int64_
  * the GEMM applies no inverse rotation.
  *
  *   c         device, [M, ldc] row-major, fp32 or bf16, ldc >= N
- * Shape rules: M % 128 == 0, N % 128 == 0, K % 128 == 0 (double block:
- * K % 256 == 0 and K <= 8192); ldc * size % 16 == 0.
+ * Shape rules: M % 128 == 0, N % 128 == 0, K % 128 == 0 (double block: also
+ * K <= 8192); ldc * size % 16 == 0.
  * The accumulation is FP32 on the tensor cores.
  */
 fp4_status_t fp4_gemm(fp4_format_t format, int double_block,

@@ -92,7 +92,6 @@ def g(**kw):
     (dict(fmt=7), 1), (dict(fmt=fp4.FP4_UFP4), 8), (dict(out=3), 1), (dict(ldc=100), 1),
     (dict(M=-128), 1), (dict(a=None), 1), (dict(ta=None), 1), (dict(db=1, fmt=fp4.FP4_MXFP4), 1),
     (dict(M=200), 2), (dict(N=192), 2), (dict(K=320), 2), (dict(K=0), 2),
-    (dict(db=1, K=384, oa=ADDR, ob=ADDR), 2),
     (dict(a=ADDR + 8), 3), (dict(ldc=260), 3),
     (dict(db=1, oa=ADDR + 8, ob=ADDR), 3), (dict(db=1, oa=ADDR, ob=ADDR + 4), 3),
     (dict(db=1, oa=None, ob=ADDR), 1), (dict(db=1, K=8448, oa=ADDR, ob=ADDR), 2),

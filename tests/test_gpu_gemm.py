@@ -144,7 +144,8 @@ def test_full_mxfp4_wgrad_down(fp4):
 
 
 @pytest.mark.parametrize("out_bf16", [False, True])
-@pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 512), (128, 256, 2048), (384, 128, 8192)])
+@pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 512), (128, 256, 2048), (384, 128, 8192),
+                                   (128, 128, 128), (256, 128, 384), (128, 256, 1152), (128, 128, 8064)])
 def test_double_block_gemm_on_oracle_operands(fp4, out_bf16, shape):
     """C = sum over 128-K chunks of s_oA * s_oB * (block-scaled partial)."""
     M, N, K = shape
