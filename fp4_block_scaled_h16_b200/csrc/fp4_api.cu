@@ -175,6 +175,7 @@ fp4_status_t fp4_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int6
     a.amax_out = reinterpret_cast<unsigned int*>(amax_out);
     a.sign_mask = sign_mask_of(rotation, seed);
     a.err = device_error_word();
+    a.wait_limit = g_wait_limit;
     if (launch_amax(a, in_dtype == FP4_IN_BF16, rot_size(rotation), axis, s) != cudaSuccess) return FP4_ERR_CUDA;
     return FP4_OK;
 }
@@ -230,6 +231,7 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
     a.tensor_id = tensor_id;
     a.sign_mask = sign_mask_of(rotation, seed);
     a.err = device_error_word();
+    a.wait_limit = g_wait_limit;
     const int rn = rot_size(rotation);
     const bool bf16 = in_dtype == FP4_IN_BF16;
     if (internal_amax) {
@@ -315,6 +317,7 @@ fp4_status_t fp4_requantize(const uint8_t* src_codes, const uint8_t* src_scales,
     a.tensor_id = tensor_id;
     a.sign_mask = sign_mask_of(rotation, seed);
     a.err = device_error_word();
+    a.wait_limit = g_wait_limit;
     a.src_codes = src_codes; a.src_scales = src_scales; a.src_outer = src_outer;
     a.src_ts = src_tensor_scale;
     a.src_fmt = src_format; a.src_db = src_double_block;

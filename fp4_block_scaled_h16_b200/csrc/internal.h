@@ -27,6 +27,7 @@ struct QuantArgs {
     uint32_t sign_mask;         // random-sign bits (0: deterministic Hadamard)
     uint32_t div_m, div_l;      // multiply-shift division by the units per line
     unsigned int* err;          // device error word (a bounded wait that ran out)
+    uint32_t wait_limit;        // polls of a bounded wait (fp4_set_wait_limit)
     // re-quantization (fp4_requantize): the source is a quantized tensor whose
     // lines are the rows of the logical [rows, cols] input; x is unused
     const uint8_t* src_codes;   // [rows, cols/2]

@@ -200,9 +200,16 @@ __device__ __forceinline__ float tensor_scale_of(float amax, int fmt) {
 }
 
 // RN(a / d) from y = RN(1/d) by one correction step: q0 = a*y, r = a - d*q0
-// (exact), q = q0 + r*y.  Exact while a, d, 1/d and the quotient are normal;
-// for d = 6 and d = 7 an exhaustive check over every normal a >= 2^-122
-// agrees with IEEE division.
+// (exact, one fused multiply-add), q = RN(q0 + r*y).  This is Markstein's
+// correction of a faithful quotient by the exact remainder (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990; "IA-64 and Elementary
+// Functions", 2000, ch. 8): with y the correctly rounded reciprocal and q0
+// within an ulp of a/d, q is the correctly rounded quotient, as long as no
+// step under- or overflows.  Callers keep a, d, 1/d and the quotient in the
+// normal range (the range tests below) and fall back to IEEE division
+// otherwise; for d = 6 and d = 7 an exhaustive check over every normal
+// a >= 2^-122 agrees with IEEE division.
 __device__ __forceinline__ float div_rcp(float a, float d, float y) {
     const float q0 = __fmul_rn(a, y);
     return __fmaf_rn(__fmaf_rn(-d, q0, a), y, q0);
@@ -278,7 +285,7 @@ struct ScaleTable {
 
 // v <- v / S per element, S and y per 16-block (SY[b] = (S_b, y_b)), on the
 // unit's pair layout: q0 = x*y, r = x - S*q0 (exact), q = q0 + r*y = RN(x/S)
-// while S and 1/S are normal (r is formed as -(S*q0 - x) so that x = -0
+// (Markstein's correction, as in div_rcp) while S and 1/S are normal (r is formed as -(S*q0 - x) so that x = -0
 // gives -0); IEEE division otherwise; S = y = 0 -> +-0.
 template <int U, int ROT>
 __device__ __forceinline__ void nv_divide(float* v, const float2* SY) {

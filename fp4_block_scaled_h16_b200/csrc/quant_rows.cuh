@@ -19,8 +19,12 @@
 // and run them again, in reverse order, to quantize -- the second read of
 // the tensor then comes mostly from L2.  Every CTA must be resident for the
 // barrier, which the cooperative launch guarantees; work that other streams
-// keep on the SMs for more than the barrier's poll budget (about 2^22 sleeps
-// of 32 ns) makes it report FP4_ERR_TIMEOUT rather than wait longer.
+// keep on the SMs for more than the barrier's poll budget (4 x the wait limit
+// of fp4_set_wait_limit, by default 2^22 sleeps of 32 ns) makes it report
+// FP4_ERR_TIMEOUT rather than wait longer.  A ring wait polls at most 16 x the
+// wait limit (2^24 by default).  Whatever way a CTA leaves, thread 0 first
+// waits (with a fixed bound) for every bulk copy it issued, so no copy lands
+// in the shared memory of a CTA that has exited.
 #pragma once
 
 #include "quant_common.cuh"
@@ -29,8 +33,11 @@
 namespace fp4 {
 
 constexpr int RQ_THREADS = 256;
-constexpr uint32_t RQ_WAIT_LIMIT = 1u << 24;
-constexpr uint32_t RQ_GRID_WAIT_LIMIT = 1u << 22;   // polls of the grid barrier (32 ns sleeps)
+constexpr uint32_t RQ_DRAIN_LIMIT = 1u << 22;       // polls of the exit drain (fixed)
+
+// ring waits: 16 x the wait limit; grid barrier: 4 x (saturating)
+__device__ __forceinline__ uint32_t ring_limit(uint32_t w) { return w >= (1u << 27) ? 0xFFFFFFFFu : w << 4; }
+__device__ __forceinline__ uint32_t grid_limit(uint32_t w) { return w >= (1u << 29) ? 0xFFFFFFFFu : w << 2; }
 
 // what a launch does: quantize with a known tensor amax, compute the rotated
 // tensor's amax only, or both in one launch (amax pass, grid barrier, quantize pass)
@@ -121,8 +128,11 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
             ne = min(st.seg_elems, (int)(a.K - e0));
         }
     };
-    // one thread fills a stage buffer: one bulk copy per line piece
+    // one thread fills a stage buffer: one bulk copy per line piece.  Fills
+    // are issued in pass order, fill v to slot v % STAGES; `issued` counts them
+    uint32_t issued = 0;
     auto issue = [&](int s, int slot) {
+        ++issued;
         int l0, nl, e0, ne;
         stage_geom(s, l0, nl, e0, ne);
         const uint32_t bytes = (uint32_t)(ne * ES);
@@ -170,7 +180,8 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
                 __threadfence();
                 atomicAdd(a.grid_count, 1u);
                 bool done = false;
-                for (uint32_t i = 0; i < RQ_GRID_WAIT_LIMIT; ++i) {
+                const uint32_t glimit = grid_limit(a.wait_limit);
+                for (uint32_t i = 0; i < glimit; ++i) {
                     if (sm100::ld_acquire_gpu(a.grid_count) >= gridDim.x) { done = true; break; }
                     __nanosleep(32);
                 }
@@ -194,7 +205,7 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
         // the warp (in the first pass of a fused launch: sends it on to the
         // pass boundary, where the whole CTA meets)
         if (!__all_sync(0xffffffffu,
-                        sm100::mbar_wait(&full[slot], (uint32_t)(it / RQ_STAGES) & 1u, RQ_WAIT_LIMIT, nullptr))) {
+                        sm100::mbar_wait(&full[slot], (uint32_t)(it / RQ_STAGES) & 1u, ring_limit(a.wait_limit), nullptr))) {
             ok = false;
             if (FUSED && it < n) { it = n - 1; continue; }
             break;
@@ -224,7 +235,7 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
         if (tid == 0 && it + RQ_STAGES - 1 < nv) {
             const int refill = (it + RQ_STAGES - 1) % RQ_STAGES;
             if (it > 0 && !sm100::mbar_wait(&empty[refill], (uint32_t)((it - 1) / RQ_STAGES) & 1u,
-                                            RQ_WAIT_LIMIT, nullptr))
+                                            ring_limit(a.wait_limit), nullptr))
                 stalled = true;
             else
                 issue(stage_of(it + RQ_STAGES - 1), refill);
@@ -314,6 +325,16 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
         }
     }
 
+    // every fill issued must land before the CTA may exit (a warp that gave up
+    // on a wait leaves fills behind it): the last fill of slot s is fill
+    // issued - 1 - ((issued - 1 - s) % STAGES), of phase (issued - 1 - s) / STAGES;
+    // all earlier fills of the slot were consumed before it was refilled
+    if (tid == 0) {
+#pragma unroll
+        for (int sl = 0; sl < RQ_STAGES; ++sl)
+            if (issued > (uint32_t)sl)
+                sm100::mbar_wait(&full[sl], ((issued - 1u - sl) / RQ_STAGES) & 1u, RQ_DRAIN_LIMIT, nullptr);
+    }
     if (!ok) {
         if (lane == 0) atomicExch(a.err, 7u);         // FP4_ERR_TIMEOUT
         return;

@@ -3,11 +3,12 @@
 // array of this library instead of a caller-provided workspace.
 //
 // Who needs it: code that runs where cudaMalloc is unavailable or forbidden --
-// inside a CUDA-graph capture that must not allocate, in a plug-in whose host
-// framework owns every device allocation, or in a real-time loop that may not
-// touch the allocator.  Such callers still own their inputs and outputs; only
-// the scratch words (the amax accumulator and a grid-barrier count) move into
-// library-owned memory.
+// a plug-in whose host framework owns every device allocation, or a
+// real-time loop that may not touch the allocator.  Such callers still own
+// their inputs and outputs; only the scratch words (the amax accumulator and
+// a grid-barrier count) move into library-owned memory.  The first call on a
+// device resolves the array's address (cudaGetSymbolAddress), so it belongs
+// before any stream capture.
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <mutex>

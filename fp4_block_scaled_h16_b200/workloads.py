@@ -108,3 +108,20 @@ def layer_linear(name, seed=0, T=TOKENS, scale_dims=1):
     W = normal(rng, (d_out, d_in), 0.02)
     dY = laplace_grad(rng, T, d_out)
     return dict(X=_bf16(X), W=_bf16(W), dY=_bf16(dY))
+
+
+# The six quantized operands of one linear, in role order: (tensor, axis,
+# stochastic rounding).  Fprop Y = X W^T takes X and W along their rows
+# (axis 1); Dgrad dX = dY W takes dY along its rows and W along its columns
+# (axis 0); Wgrad dW = dY^T X takes dY and X along their columns (axis 0),
+# with stochastic rounding ("Pre-addestramento ... con MXFP4", Metodologia:
+# the three GEMMs of every linear).
+LAYER_OPERANDS = (("X", 1, False), ("W", 1, False), ("dY", 1, False),
+                  ("W", 0, False), ("dY", 0, True), ("X", 0, True))
+# The three GEMMs: (name, operand role of A, operand role of B, bf16 output?)
+LAYER_GEMMS = (("fprop", 0, 1, True), ("dgrad", 2, 3, True), ("wgrad", 4, 5, False))
+
+
+def layer_tensor_id(linear_index: int, role: int) -> int:
+    """Stochastic-rounding stream of one operand: 16 * linear + role."""
+    return 16 * linear_index + role

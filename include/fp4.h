@@ -26,8 +26,10 @@
  *     stream).  Calls are asynchronous on it: outputs are valid once the
  *     stream has reached the call.
  *   - Argument, shape and alignment errors are returned synchronously and
- *     nothing is launched.  A failed launch returns FP4_ERR_CUDA.  Device-side
- *     timeouts of the GEMM pipeline are reported by fp4_last_error().
+ *     nothing is launched.  A failed launch returns FP4_ERR_CUDA.  A bounded
+ *     device-side wait that ran out (a GEMM pipeline hand-off, a ring wait
+ *     or the grid barrier of the row-axis quantizer) is reported by
+ *     fp4_last_error() as FP4_ERR_TIMEOUT.
  *   - Pointers to tensor data must be 16-byte aligned.
  *
  * Quantized tensor ("K-major view")
@@ -277,9 +279,11 @@ fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
 
 /*
  * fp4_last_error -- synchronizes `stream` and returns (and clears) the device
- * error word the kernels set: FP4_ERR_TIMEOUT when a bounded wait in the GEMM
- * pipeline gave up (the kernel then abandons its tile and exits cleanly),
- * FP4_OK otherwise, FP4_ERR_CUDA if the synchronization failed.
+ * error word the kernels set: FP4_ERR_TIMEOUT when a bounded wait gave up (a
+ * GEMM pipeline hand-off, a quantizer ring wait or its grid barrier; the kernel
+ * then lets its own copies in flight land, frees what it holds and exits; its
+ * outputs are not valid), FP4_OK otherwise, FP4_ERR_CUDA if the
+ * synchronization failed.
  */
 fp4_status_t fp4_last_error(void* stream);
 
@@ -287,9 +291,13 @@ fp4_status_t fp4_last_error(void* stream);
 const char* fp4_status_string(fp4_status_t status);
 
 /*
- * fp4_set_wait_limit -- iteration limit of every bounded device-side wait
- * (default 2^20 polls, far above any legitimate wait).  A test can lower it to
- * make a wait run out without hanging the GPU.  0 restores the default.
+ * fp4_set_wait_limit -- iteration limit of the bounded device-side waits of
+ * later calls (default 2^20 polls, far above any legitimate wait): a GEMM
+ * hand-off polls at most this many times, a quantizer ring wait 16 times as
+ * many and the quantizer's grid barrier 4 times as many (32 ns sleeps).  A
+ * test can lower it to make a wait run out without hanging the GPU.  0
+ * restores the default.  Process-wide; not synchronized with calls in flight
+ * on other host threads.
  */
 void fp4_set_wait_limit(uint32_t polls);
 

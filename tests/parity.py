@@ -32,6 +32,16 @@ def untile(buf: np.ndarray, L: int, K: int, fmt: int) -> np.ndarray:
     return buf[tiled_offsets(L, K, fmt)]
 
 
+def untile_lines(buf: np.ndarray, lines: np.ndarray, K: int, fmt: int) -> np.ndarray:
+    """[len(lines), K/blk] scale bytes of the given lines from a tiled buffer."""
+    blk = FMT_BLK[fmt]
+    nb = K // blk
+    nb4 = (nb + 3) // 4
+    l = np.asarray(lines, dtype=np.int64)[:, None]
+    b = np.arange(nb, dtype=np.int64)[None, :]
+    return buf[((l // 128) * nb4 + b // 4) * 512 + (l % 32) * 16 + ((l % 128) // 32) * 4 + (b % 4)]
+
+
 def tile(rowmajor: np.ndarray, fmt: int, nbytes: int) -> np.ndarray:
     L, nb = rowmajor.shape
     K = nb * FMT_BLK[fmt]

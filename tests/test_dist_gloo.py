@@ -51,3 +51,16 @@ def test_sharded_amax_quantization_equals_unsharded():
     out = mp.get_context("spawn").Manager().dict()
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
     assert dict(out) == {0: 1, 1: 1}
+
+
+class _FakeFp4:
+    """Stands in for the binding in a host-logic test: only the constants."""
+    FP4_RTNE, FP4_SR = 0, 1
+
+
+def test_row_shard_helper_refuses_stochastic_rounding():
+    # the SR counter of a shard is shard-local, so sharded SR is not the
+    # unsharded result; the helper must say so before launching anything
+    from fp4_block_scaled_h16_b200.dist import quantize_row_shard
+    with pytest.raises(ValueError, match="stochastic rounding"):
+        quantize_row_shard(_FakeFp4, torch.zeros((4, 16)), fmt=1, rounding=_FakeFp4.FP4_SR)

@@ -1,4 +1,5 @@
-"""Failure detection of the GEMM pipelines without a GPU fault.
+"""Failure detection of the GEMM pipelines and the one-launch quantizer
+without a GPU fault.
 
 Every hand-off inside the GEMM kernels (TMA producer -> MMA issuer ->
 epilogue, and the double-block GEMM's partial and outer-scale buffers) is an
@@ -57,3 +58,33 @@ def test_gemm_wait_timeout_is_reported_and_recoverable(fp4, fmt, double_block, o
     assert fp4.fp4_last_error() == fp4.FP4_OK
     assert torch.equal(before.view(torch.int16 if out == "BF16" else torch.int32),
                        after.view(torch.int16 if out == "BF16" else torch.int32))
+
+
+# The one-launch quantizer (tensor amax pass, grid barrier, quantize pass)
+# waits on its shared-memory ring and on the grid barrier; both budgets follow
+# the wait limit (16 x and 4 x).  At one poll the barrier runs out long before
+# every CTA has finished the amax pass of a 8192 x 4096 tensor.  The kernel
+# lets its own bulk copies land before it exits; the next call at the default
+# limit must give the bytes a call before the timeout gave.
+@pytest.mark.parametrize("fmt,rounding,rotation", [("NVFP4", 0, 1), ("UFP4", 1, 3)])
+def test_one_launch_quantizer_wait_timeout_is_reported_and_recoverable(fp4, fmt, rounding, rotation):
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn((8192, 4096), generator=g).to(torch.bfloat16).cuda()
+    kw = dict(fmt=getattr(fp4, "FP4_" + fmt), rounding=rounding, rotation=rotation, axis=1, seed=3, tensor_id=2)
+    before = fp4.quantize(x, **kw)
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+
+    fp4.fp4_set_wait_limit(1)
+    try:
+        fp4.quantize(x, **kw)
+        status = fp4.fp4_last_error()
+    finally:
+        fp4.fp4_set_wait_limit(0)
+    assert status == fp4.FP4_ERR_TIMEOUT, fp4.fp4_status_string(status)
+
+    after = fp4.quantize(x, **kw)
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    for key in ("codes", "tensor_scale"):
+        assert torch.equal(before[key].view(torch.uint8), after[key].view(torch.uint8)), key
+    n = fp4.fp4_scales_bytes(8192, 4096, kw["fmt"])
+    assert torch.equal(before["scales"][:n], after["scales"][:n])

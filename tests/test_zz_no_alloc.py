@@ -1,6 +1,8 @@
 """fp4_quantize_noalloc -- the entry point for callers that cannot allocate
-device memory (its scratch is a static array inside libfp4.so) -- must give
-exactly what fp4_quantize with a caller workspace gives, call after call.
+device memory (a plug-in whose host framework owns every device allocation, a
+loop that may not touch the allocator): its scratch is a static array inside
+libfp4.so.  It must give exactly what fp4_quantize with a caller workspace
+gives, call after call, and both must agree with the CPU oracle.
 
 Collected last on purpose: the static scratch keeps the previous call's
 contents, so this must hold both in a fresh process and after every other
@@ -9,6 +11,8 @@ test has used the library.
 import numpy as np
 import pytest
 import torch
+
+from parity import assert_quant_equal, oracle_quantize, untile
 
 pytestmark = pytest.mark.gpu
 
@@ -63,6 +67,13 @@ def test_noalloc_matches_workspace_path_two_calls(fp4, fmt, rounding, rotation, 
         a = via_workspace(fp4, x, fmt, rounding, rotation, axis, 11, 5 + i)
         b = via_noalloc(fp4, x, fmt, rounding, rotation, axis, 11, 5 + i)
         same(fp4, a, b)
+        # and the static-scratch result is the oracle's, bit for bit
+        o = oracle_quantize(x.cpu(), fmt=fmt, rounding=rounding, rotation=rotation, axis=axis, seed=11,
+                            tensor_id=5 + i)
+        g = dict(codes=b["codes"].cpu().numpy(),
+                 scales=untile(b["scales"].cpu().numpy(), b["lines"], b["K"], fmt),
+                 outer=None, tensor_scale=float(b["tensor_scale"].cpu()[0]))
+        assert_quant_equal(g, o, what="noalloc call %d" % i)
 
 
 def test_noalloc_rejects_mxfp4_and_bad_args(fp4):
