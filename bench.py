@@ -1,23 +1,28 @@
 #!/usr/bin/env python
 """Benchmark of the block-scaled FP4 hot path on B200.
 
-One step = one pass of the whole path over one batch: the NVFP4 Fprop of the
-Llama-3.1-8B QKV projection at 8192 tokens -- rotated-tensor amax and fused
-H16-rotate/scale/round/pack quantization of X [8192, 4096] and of
-W [6144, 4096] (bf16), then the block-scaled FP4 GEMM Y = X W^T
-(8192 x 6144 x 4096, bf16 out).
+One step = one pass of the whole path over the linears of one Llama-3.1-8B
+decoder layer at 8192 tokens: QKV 4096 -> 6144, O 4096 -> 4096, fused
+gate+up 4096 -> 28672, down 14336 -> 4096.  For each linear the six operands
+of its Fprop, Dgrad and Wgrad GEMMs are quantized to NVFP4 with H16 (rotated
+tensor amax, rotate, block scale, round, pack; stochastic rounding on the
+Wgrad operands; the Dgrad and Wgrad operands along the transposed axis) and
+the three block-scaled FP4 GEMMs run: 24 quantize calls and 12 GEMMs,
+10.72 TFLOP of GEMM work per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp4|reference]
 
-Prints one JSON line (rank 0).  Multi-GPU: one process per GPU under torchrun,
-each rank runs its own independent problem (weak scaling, no collective on the
-data path); the time is the max over ranks.
+Prints one JSON line (rank 0).  `value` is the step's GEMM FLOP over the whole
+step time (quantization included).  Multi-GPU: one process per GPU under
+torchrun, each rank runs its own independent layer (weak scaling, no
+collective on the data path); the time is the max over ranks.
 """
 from __future__ import annotations
 
 import argparse
 import json
 import os
+import platform
 import statistics
 import sys
 import threading
@@ -32,15 +37,16 @@ sys.path.insert(0, ROOT)
 from fp4_block_scaled_h16_b200 import workloads  # noqa: E402
 
 METRIC = "FP4 quantize GB/s and block-scaled FP4 GEMM TFLOPS (% of B200 roofline)"
-M, N, K = workloads.TOKENS, workloads.QKV_OUT, workloads.HIDDEN
-WORKLOAD = "nvfp4_fprop_qkv_%dx%dx%d" % (M, N, K)
-GEMM_FLOP = 2.0 * M * N * K
+WORKLOAD = "llama31_8b_layer_linears_t8192_nvfp4_h16"
+T = workloads.TOKENS
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gemm_kernel
-# launch on this workload, from one ncu capture of the current kernel: 36.3 MB
-# read (the 33 MB of operands cross DRAM once) and 49.5 MB written (the rest of
-# the 100.7 MB of C was still in L2 when the kernel ended)
-GEMM_TRAFFIC_BYTES = 36_268_032 + 49_481_728
+OPERANDS = workloads.LAYER_OPERANDS
+GEMMS = workloads.LAYER_GEMMS
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per gemm_kernel
+# launch, averaged over the 12 GEMM launches of one layer step, from one ncu
+# capture of the current kernel (profiles/gemm_layer_llama8b_t8192.md); None
+# until that capture exists
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = None
 
 
 class L2Flush:
@@ -56,10 +62,6 @@ class L2Flush:
     def __call__(self):
         self.w.zero_()
         torch.amax(self.r, dim=0, out=self.sink)
-# algorithmic bytes per element (bf16 in): amax pass reads 2 B; the quantize
-# pass reads 2 B and writes 0.5 B of codes + 1/16 B of E4M3 scale
-AMAX_BPE = 2.0
-QUANT_BPE = 2.0 + 0.5 + 1.0 / 16.0
 
 
 def measured_peaks():
@@ -70,6 +72,17 @@ def measured_peaks():
         return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained"),
                     src="measured")
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
 
 class ClockSampler:
@@ -118,50 +131,225 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": names}
 
 
+def qbytes(numel, elem_bytes, fmt, db=False, reads=1):
+    """Algorithmic bytes of one quantize call: the input read `reads` times,
+    codes + scales (+ outer scales) written."""
+    blk = 32 if fmt == 0 else 16
+    return reads * numel * elem_bytes + numel / 2 + numel / blk + (numel / 128 * 4 if db else 0)
+
+
+def quantize_kernels(axis, internal_amax):
+    """Kernels one fp4_quantize call launches: the row axis runs the amax and
+    quantize passes as one cooperative kernel; axis 0 runs an amax kernel then
+    the quantize kernel; with a given amax (or MXFP4 / double block) one."""
+    return 2 if (internal_amax and axis == 0) else 1
+
+
 # ------------------------------------------------------------------------ GPU arm
 
+class LayerStep:
+    """Device buffers and the step of the layer workload: per linear, the six
+    NVFP4 + H16 operands and the Fprop, Dgrad and Wgrad GEMMs."""
+
+    def __init__(self, fp4, device, seed=0, fmt=None, host=None):
+        self.fp4 = fp4
+        self.fmt = fp4.FP4_NVFP4 if fmt is None else fmt
+        self.device = device
+        self.linears = []
+        self.flop = 0.0
+        self.quant_bytes = 0.0
+        self.ws = torch.empty(256, dtype=torch.uint8, device=device)
+        self.launches = 0
+        for index, (name, d_in, d_out, _) in enumerate(workloads.LAYER_LINEARS):
+            d = host[index] if host is not None else workloads.layer_linear(name, seed=seed)
+            t = {k: v.to(device) for k, v in d.items()}
+            qs, calls = [], []
+            for role, (tn, axis, sr) in enumerate(OPERANDS):
+                R, C = t[tn].shape
+                L, K = (R, C) if axis == 1 else (C, R)
+                qs.append(fp4.alloc_qtensor(L, K, self.fmt, device=device))
+                calls.append(dict(x=tn, axis=axis, rounding=fp4.FP4_SR if sr else fp4.FP4_RTNE,
+                                  tensor_id=workloads.layer_tensor_id(index, role), name="%s_ax%d" % (tn, axis)))
+                self.quant_bytes += qbytes(R * C, 2, self.fmt, reads=2)
+                self.launches += quantize_kernels(axis, True)
+            outs = []
+            for gname, ra, rb, bf16 in GEMMS:
+                M, N, K = qs[ra]["lines"], qs[rb]["lines"], qs[ra]["K"]
+                outs.append(torch.empty((M, N), dtype=torch.bfloat16 if bf16 else torch.float32, device=device))
+                self.flop += 2.0 * M * N * K
+                self.launches += 1
+            self.linears.append(dict(name=name, t=t, qs=qs, calls=calls, outs=outs))
+
+    def quantize(self, lin, role):
+        c = lin["calls"][role]
+        self.fp4.quantize(lin["t"][c["x"]], self.fmt, c["rounding"], self.fp4.FP4_ROT_H16, axis=c["axis"],
+                          seed=0, tensor_id=c["tensor_id"], out=lin["qs"][role], workspace=self.ws)
+
+    def gemm(self, lin, g):
+        _, ra, rb, bf16 = GEMMS[g]
+        self.fp4.gemm(lin["qs"][ra], lin["qs"][rb], self.fp4.FP4_OUT_BF16 if bf16 else self.fp4.FP4_OUT_F32,
+                      out=lin["outs"][g])
+
+    def calls(self):
+        """The step's calls in order: (kind, linear name, call name, fn)."""
+        out = []
+        for lin in self.linears:
+            for role in range(len(OPERANDS)):
+                kind = "quant_rows" if lin["calls"][role]["axis"] == 1 else "quant_cols"
+                out.append((kind, lin["name"], lin["calls"][role]["name"], role, lin))
+            for g in range(len(GEMMS)):
+                out.append(("gemm", lin["name"], GEMMS[g][0], g, lin))
+        return out
+
+    def run_call(self, c):
+        kind, _, _, i, lin = c
+        if kind == "gemm":
+            self.gemm(lin, i)
+        else:
+            self.quantize(lin, i)
+
+    def step(self):
+        for lin in self.linears:
+            for role in range(len(OPERANDS)):
+                self.quantize(lin, role)
+            for g in range(len(GEMMS)):
+                self.gemm(lin, g)
+
+
+def time_steps(fn, flush, n):
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    for e in evs:
+        flush()
+        e[0].record()
+        fn()
+        e[1].record()
+    torch.cuda.synchronize()
+    return [e[0].elapsed_time(e[1]) for e in evs]
+
+
+def _median_ms(fn, flush, reps):
+    """Median CUDA-event time of fn() over reps runs, L2 flushed before each."""
+    fn()
+    return statistics.median(time_steps(fn, flush, reps))
+
+
+def per_call_split(layer, flush, reps, peaks):
+    """Each call of the step timed on its own (events between the calls of
+    eager steps), with its algorithmic rate and fraction of peak."""
+    calls = layer.calls()
+    ms = [[] for _ in calls]
+    for _ in range(reps):
+        flush()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        evs[0].record()
+        for i, c in enumerate(calls):
+            layer.run_call(c)
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        for i in range(len(calls)):
+            ms[i].append(evs[i].elapsed_time(evs[i + 1]))
+    fp4_peak = peaks["bf16"] * 4.0
+    table, fam = {}, {}
+    for c, m in zip(calls, ms):
+        kind, lname, cname, i, lin = c
+        t = statistics.mean(m)
+        if kind == "gemm":
+            _, ra, rb, _ = GEMMS[i]
+            M, N, K = lin["qs"][ra]["lines"], lin["qs"][rb]["lines"], lin["qs"][ra]["K"]
+            work = 2.0 * M * N * K
+            e = {"ms": t, "tflops": work / (t * 1e-3) / 1e12, "frac_fp4": work / (t * 1e-3) / 1e12 / fp4_peak,
+                 "shape": [M, N, K], "launches": 1}
+        else:
+            x = lin["t"][lin["calls"][i]["x"]]
+            work = qbytes(x.numel(), 2, layer.fmt, reads=2)
+            axis = lin["calls"][i]["axis"]
+            e = {"ms": t, "gbs": work / (t * 1e6), "frac_hbm": work / (t * 1e6) / peaks["hbm"],
+                 "bytes": "2 reads (amax pass + quantize)", "launches": quantize_kernels(axis, True),
+                 "rounding": "SR" if lin["calls"][i]["rounding"] else "RTNE"}
+        table.setdefault(lname, {})[cname] = e
+        f = fam.setdefault(kind, {"ms": 0.0, "work": 0.0, "launches": 0})
+        f["ms"] += t
+        f["work"] += work
+        f["launches"] += e["launches"]
+    for kind, f in fam.items():
+        if kind == "gemm":
+            f["tflops"] = f["work"] / (f["ms"] * 1e-3) / 1e12
+            f["frac_fp4"] = f["tflops"] / fp4_peak
+        else:
+            f["gbs"] = f["work"] / (f["ms"] * 1e6)
+            f["frac_hbm"] = f["gbs"] / peaks["hbm"]
+    return table, fam
+
+
 class Fprop:
-    """Device buffers and the step of the NVFP4 Fprop workload."""
+    """The NVFP4 Fprop of the QKV projection (8192 x 6144 x 4096): quantize X
+    and W (each with its tensor amax, one launch), then the GEMM."""
 
     def __init__(self, fp4, X, W, device):
         self.fp4 = fp4
         self.X, self.W = X.to(device), W.to(device)
+        M, K = self.X.shape
+        N = self.W.shape[0]
+        self.shape = (M, N, K)
         self.qx = fp4.alloc_qtensor(M, K, fp4.FP4_NVFP4, device=device)
         self.qw = fp4.alloc_qtensor(N, K, fp4.FP4_NVFP4, device=device)
-        self.ax = torch.empty(1, dtype=torch.float32, device=device)
-        ws = fp4.fp4_quantize_workspace_size(fp4.FP4_NVFP4, False, False)
-        self.wsx = torch.empty(ws, dtype=torch.uint8, device=device)
-        self.wsw = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(256, dtype=torch.uint8, device=device)
         self.C = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-        # quantize X (amax pass + quantize pass in one launch), the same for W, GEMM
-        self.launches_per_step = 3
 
-    def quant(self, x, q, ws):
+    def step(self):
         f = self.fp4
-        f.quantize(x, f.FP4_NVFP4, f.FP4_RTNE, f.FP4_ROT_H16, axis=1, out=q, workspace=ws)
-
-    def gemm(self):
-        self.fp4.gemm(self.qx, self.qw, self.fp4.FP4_OUT_BF16, out=self.C)
-
-    def step(self, ev=None):
-        if ev:
-            ev[0].record()
-        self.quant(self.X, self.qx, self.wsx)
-        if ev:
-            ev[1].record()
-        self.quant(self.W, self.qw, self.wsw)
-        if ev:
-            ev[2].record()
-        self.gemm()
-        if ev:
-            ev[3].record()
+        f.quantize(self.X, f.FP4_NVFP4, f.FP4_RTNE, f.FP4_ROT_H16, axis=1, out=self.qx, workspace=self.ws)
+        f.quantize(self.W, f.FP4_NVFP4, f.FP4_RTNE, f.FP4_ROT_H16, axis=1, out=self.qw, workspace=self.ws)
+        f.gemm(self.qx, self.qw, f.FP4_OUT_BF16, out=self.C)
 
 
-def run_gpu(args, rank, world, device):
+def fprop_component(fp4, device, flush, peaks, reps):
+    d = workloads.nvfp4_fprop_qkv(seed=0)
+    w = Fprop(fp4, d["X"], d["W"], device)
+    M, N, K = w.shape
+    step = _median_ms(w.step, flush, reps)
+    gemm = _median_ms(lambda: fp4.gemm(w.qx, w.qw, fp4.FP4_OUT_BF16, out=w.C), flush, reps)
+    flop = 2.0 * M * N * K
+    out = {"workload": "nvfp4_fprop_qkv_%dx%dx%d" % (M, N, K),
+           "step_ms": step, "step_tflops": flop / (step * 1e-3) / 1e12,
+           "gemm_ms": gemm, "gemm_tflops": flop / (gemm * 1e-3) / 1e12,
+           "gemm_frac_fp4": flop / (gemm * 1e-3) / 1e12 / (4 * peaks["bf16"])}
+    # context ratio ("Ripensare il Bias di Shrinkage...", Efficienza: fused
+    # RHT + quantization about 1.06-1.07x the quantization alone, unfused
+    # 1.4-1.6x, on SM90 / SM100 at sizes the pages do not state): NVFP4 of X
+    # with the random-sign H16 fused, without a rotation, and as a separate
+    # rotation kernel (bf16 out) followed by the quantizer without rotation
+    qx, ws = w.qx, w.ws
+    Xr = torch.empty_like(w.X)
+    NV, RT = fp4.FP4_NVFP4, fp4.FP4_RTNE
+    fused = _median_ms(lambda: fp4.quantize(w.X, NV, RT, fp4.FP4_ROT_RH16, axis=1, seed=5, out=qx, workspace=ws),
+                       flush, reps)
+    none = _median_ms(lambda: fp4.quantize(w.X, NV, RT, fp4.FP4_ROT_NONE, axis=1, out=qx, workspace=ws),
+                      flush, reps)
+
+    def unfused():
+        fp4.rotate(w.X, fp4.FP4_ROT_RH16, seed=5, out=Xr)
+        fp4.quantize(Xr, NV, RT, fp4.FP4_ROT_NONE, axis=1, out=qx, workspace=ws)
+
+    unf = _median_ms(unfused, flush, reps)
+    rot_only = _median_ms(lambda: fp4.rotate(w.X, fp4.FP4_ROT_RH16, seed=5, out=Xr), flush, reps)
+    out["context_ratio"] = {
+        "tensor": "X bf16 %dx%d, NVFP4, RTNE, internal tensor amax (one launch)" % (M, K),
+        "fused_rh16_ms": fused, "no_rotation_ms": none, "unfused_rotate_then_quantize_ms": unf,
+        "rotate_kernel_alone_ms": rot_only,
+        "fused_over_none": fused / none, "unfused_over_none": unf / none,
+        "pages": "fused ~1.06-1.07x, unfused ~1.4-1.6x of standalone quantization (SM90/SM100; sizes not stated)"}
+    del w, Xr
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_gpu(args, rank, world, device, host):
+    """The timed layer steps, the per-call split and the end-to-end steps;
+    `host` holds the layer's inputs in host memory (layer_host_data)."""
     from fp4_block_scaled_h16_b200 import fp4
     peaks = measured_peaks()
-    d = workloads.nvfp4_fprop_qkv(seed=rank)
-    w = Fprop(fp4, d["X"], d["W"], device)
+    layer = LayerStep(fp4, device, seed=rank, host=host)
     flush = L2Flush(device)
 
     def barrier():
@@ -169,81 +357,49 @@ def run_gpu(args, rank, world, device):
             torch.distributed.barrier()
 
     for _ in range(args.warmup):
-        w.step()
+        layer.step()
     torch.cuda.synchronize()
     assert fp4.fp4_last_error() == fp4.FP4_OK
 
-    # optionally the step as one CUDA graph (its 3 kernels and 2 workspace
-    # memsets), captured on a side stream after the eager warm-up
     graph = None
     if args.graph:
+        # the step as one CUDA graph (its kernels and workspace memsets),
+        # captured on a side stream after the eager warm-up
         side = torch.cuda.Stream(device)
         side.wait_stream(torch.cuda.current_stream(device))
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.stream(side):
-            w.step()
+            layer.step()
             torch.cuda.synchronize()
             with torch.cuda.graph(graph, stream=side):
-                w.step()
+                layer.step()
         torch.cuda.current_stream(device).wait_stream(side)
         torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(device.index) as clocks:
-        for i in range(args.steps):
-            flush()                       # L2 flush, outside the timed events
-            evs[i][0].record()
-            if graph is not None:
-                graph.replay()
-            else:
-                w.step()
-            evs[i][1].record()
-        torch.cuda.synchronize()
+        step_ms = time_steps(graph.replay if graph is not None else layer.step, flush, args.steps)
     barrier()
-    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_ms = sum(step_ms)
     status = fp4.fp4_last_error()
 
-    # the step's kernels one by one (eager, events between them)
-    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(max(3, min(args.steps, 20)))]
-    for e in evk:
-        flush()
-        w.step(e)
-    torch.cuda.synchronize()
-    qx = [e[0].elapsed_time(e[1]) for e in evk]
-    qw = [e[1].elapsed_time(e[2]) for e in evk]
-    gm = [e[2].elapsed_time(e[3]) for e in evk]
+    table, fam = per_call_split(layer, flush, max(3, min(args.steps, 10)), peaks)
 
-    # the two passes as separate kernels (fp4_amax, then fp4_quantize given the
-    # amax), timed on a second pass: each kernel against its own bytes
-    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    amax_ms, quant_ms = [], []
-    for _ in range(max(3, min(args.steps, 20))):
-        flush()
-        ev_a[0].record()
-        fp4.fp4_amax(w.X, fp4.FP4_IN_BF16, M, K, K, fp4.FP4_ROT_H16, 1, 0, w.ax)
-        ev_a[1].record()
-        fp4.quantize(w.X, fp4.FP4_NVFP4, fp4.FP4_RTNE, fp4.FP4_ROT_H16, axis=1, tensor_amax=w.ax, out=w.qx)
-        ev_a[2].record()
-        torch.cuda.synchronize()
-        amax_ms.append(ev_a[0].elapsed_time(ev_a[1]))
-        quant_ms.append(ev_a[1].elapsed_time(ev_a[2]))
-
-    # end to end through the public API: every step copies its inputs from
-    # pinned host memory and its whole result back.  Two sets of device
-    # buffers and three streams (host->device, compute, device->host) let
-    # step i+1's inputs and step i-1's result cross PCIe, in both directions,
-    # while step i computes; the timed region spans all the steps.
-    e2e_steps = max(4, min(args.steps, 20))
-    hX = d["X"].pin_memory()
-    hW = d["W"].pin_memory()
-    hC = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    slots = [w, Fprop(fp4, d["X"], d["W"], device)]
+    # end to end through the public API: every step copies its inputs (X, W and
+    # dY of the four linears) from pinned host memory and its results (the 12
+    # GEMM outputs) back.  Two sets of device buffers on three streams
+    # (host->device, compute, device->host) let step i+1's inputs and step
+    # i-1's results cross PCIe while step i computes.
+    e2e_steps = 4
+    hin = [{k: v.pin_memory() for k, v in h.items()} for h in host]
+    hout = [[[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in lin["outs"]] for lin in layer.linears]
+            for _ in range(2)]
+    second = LayerStep(fp4, device, host=hin)
+    slots = [layer, second]
     s_in, s_run, s_out = (torch.cuda.Stream(device) for _ in range(3))
     ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "run", "out")}
-    for k in ev:                                  # every slot starts free
+    for k in ev:
         for e in ev[k]:
             e.record()
     torch.cuda.synchronize()
@@ -251,126 +407,107 @@ def run_gpu(args, rank, world, device):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s_in)
-    for _ in (s_run, s_out):
-        _.wait_stream(s_in)
+    for st in (s_run, s_out):
+        st.wait_stream(s_in)
     for i in range(e2e_steps):
         k = i % 2
         f = slots[k]
         with torch.cuda.stream(s_in):
-            s_in.wait_event(ev["run"][k])         # step i-2 is done reading this slot
-            f.X.copy_(hX, non_blocking=True)
-            f.W.copy_(hW, non_blocking=True)
+            s_in.wait_event(ev["run"][k])          # step i-2 is done reading this slot
+            for lin, h in zip(f.linears, hin):
+                for name, t in lin["t"].items():
+                    t.copy_(h[name], non_blocking=True)
             ev["in"][k].record(s_in)
         with torch.cuda.stream(s_run):
             s_run.wait_event(ev["in"][k])
-            s_run.wait_event(ev["out"][k])        # step i-2's result has left this slot
+            s_run.wait_event(ev["out"][k])         # step i-2's results have left this slot
             f.step()
             ev["run"][k].record(s_run)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev["run"][k])
-            hC[k].copy_(f.C, non_blocking=True)
+            for lin, h in zip(f.linears, hout[k]):
+                for o, ho in zip(lin["outs"], h):
+                    ho.copy_(o, non_blocking=True)
             ev["out"][k].record(s_out)
     s_out.wait_stream(s_in)
     s_out.wait_stream(s_run)
     e1.record(s_out)
     torch.cuda.synchronize()
-    e2e_ms = [e0.elapsed_time(e1) / e2e_steps]
-    del slots[1]
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = sum(v.numel() * v.element_size() for h in hin for v in h.values())
+    d2h = sum(o.numel() * o.element_size() for lin in layer.linears for o in lin["outs"])
+    del slots, second, hout
+    torch.cuda.empty_cache()
 
-    t = torch.tensor([total_ms, statistics.mean(e2e_ms)], dtype=torch.float64, device=device)
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     total_max, e2e_max = float(t[0]), float(t[1])
     if rank != 0:
-        return None
+        return None, layer
 
     ms_per_step = total_max / args.steps
-    value = world * args.steps * GEMM_FLOP / (total_max * 1e-3) / 1e12
-    gemm_ms = statistics.mean(gm)
-    fp4_peak = peaks["bf16"] * 4.0      # nominal dense fp4 / bf16 ratio (9 / 2.25 PFLOP/s)
-    achieved = GEMM_FLOP / (gemm_ms * 1e-3) / 1e12
-    bpe_x = M * K
-    comp = {
-        "amax_X": {"ms": statistics.mean(amax_ms), "gbs": AMAX_BPE * bpe_x / (statistics.mean(amax_ms) * 1e6),
-                   "kernel": "fp4_amax alone"},
-        "quantize_X": {"ms": statistics.mean(quant_ms), "gbs": QUANT_BPE * bpe_x / (statistics.mean(quant_ms) * 1e6),
-                       "kernel": "fp4_quantize given the amax"},
-        "amax+quantize_X": {"ms": statistics.mean(qx), "gbs_2read": (AMAX_BPE + QUANT_BPE) * M * K / (statistics.mean(qx) * 1e6),
-                            "gbs_1read": QUANT_BPE * M * K / (statistics.mean(qx) * 1e6),
-                            "kernel": "fp4_quantize, internal amax: one launch (as timed in the step)"},
-        "amax+quantize_W": {"ms": statistics.mean(qw), "gbs_2read": (AMAX_BPE + QUANT_BPE) * N * K / (statistics.mean(qw) * 1e6),
-                            "gbs_1read": QUANT_BPE * N * K / (statistics.mean(qw) * 1e6),
-                            "kernel": "fp4_quantize, internal amax: one launch (as timed in the step)"},
-        "gemm": {"ms": gemm_ms, "tflops": achieved},
-    }
-    for k in ("amax_X", "quantize_X"):
-        comp[k]["frac_hbm"] = comp[k]["gbs"] / peaks["hbm"]
-    for k in ("amax+quantize_X", "amax+quantize_W"):
-        comp[k]["frac_hbm"] = comp[k]["gbs_2read"] / peaks["hbm"]
-        comp[k]["frac_hbm_1read"] = comp[k]["gbs_1read"] / peaks["hbm"]
-    comp["gemm"]["frac_fp4"] = achieved / fp4_peak
+    value = world * args.steps * layer.flop / (total_max * 1e-3) / 1e12
+    fp4_peak = peaks["bf16"] * 4.0
+    # the dominant kernel family of the step, by time
+    dom = max(fam, key=lambda k: fam[k]["ms"])
+    f = fam[dom]
+    if dom == "gemm":
+        roof = {"bound": "tensor", "kernel": "gemm_kernel (NVFP4, 12 launches per step)",
+                "achieved": round(f["tflops"], 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                "frac": round(f["tflops"] / fp4_peak, 4), "traffic": GEMM_TRAFFIC_BYTES_PER_LAUNCH,
+                "achieved_is": "GEMM FLOP of the step / summed mean event time of its 12 GEMM launches",
+                "peak_is": "%s bf16 burst %.1f TFLOP/s x 4 (nominal fp4 / bf16 ratio)" % (peaks["src"], peaks["bf16"])}
+    else:
+        roof = {"bound": "hbm", "kernel": ("quant_rows_kernel" if dom == "quant_rows" else
+                                           "quant_cols_kernel (amax + quantize)") + ", 12 calls per step",
+                "achieved": round(f["gbs"], 1), "peak": round(peaks["hbm"], 1), "unit": "GB/s",
+                "frac": round(f["gbs"] / peaks["hbm"], 4), "traffic": None,
+                "achieved_is": "algorithmic bytes (input read twice: amax pass + quantize; codes and "
+                               "scales written) / summed mean event time",
+                "peak_is": "%s HBM copy bandwidth" % peaks["src"]}
+    roof["families"] = {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                        for k, v in fam.items()}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e2m1, e4m3 scales) -> f32 accumulate; quantizer f32",
-        "data": "synthetic (seeded: X N(0,1) with 8 outlier channels x64, W N(0,0.02); bf16)",
-        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "format": "NVFP4",
-                   "rotation": "H16", "rounding": "RTNE", "out": "bf16",
-                   "value_is": "GEMM FLOP of the step / whole step time (quantize X and W, each with its tensor amax, + GEMM)",
-                   "l2": "flushed between steps (256 MiB write, then 256 MiB read, outside the timed events)",
+        "data": "synthetic (seeded: activations N(0,1) with 8 outlier channels x64 or SwiGLU N(0,1)*silu(N(0,1)), "
+                "W N(0,0.02), dY Laplace(0,1e-3); bf16)",
+        "config": {"workload": WORKLOAD, "tokens": T,
+                   "linears": {n: [d_in, d_out] for n, d_in, d_out, _ in workloads.LAYER_LINEARS},
+                   "format": "NVFP4", "rotation": "H16 on all three GEMMs",
+                   "rounding": "RTNE; SR on the Wgrad operands", "out": "bf16 (Fprop, Dgrad), f32 (Wgrad)",
+                   "gemm_flop_per_step": layer.flop,
+                   "value_is": "GEMM FLOP of the step / whole step time (24 quantize calls, each with its "
+                               "tensor amax, + 12 GEMMs)",
+                   "l2": "flushed before every step (256 MiB write, then 256 MiB read, outside the timed "
+                         "events); the step's 1.6 GB of inputs exceed L2",
                    "launch": "the step replayed as one CUDA graph" if args.graph else "eager launches",
-                   "parallelism": "independent problem per GPU" if world > 1 else "single GPU"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_kernel (NVFP4, 128x256 tile)",
-                     "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / fp4_peak, 4), "traffic": GEMM_TRAFFIC_BYTES,
-                     "traffic_is": "ncu dram read + write bytes of one launch (algorithmic: 33.0 MB read, 100.7 MB written)",
-                     "peak_is": "%s bf16 burst %.1f TFLOP/s x 4 (nominal fp4/bf16)" % (peaks["src"], peaks["bf16"])},
-        "components": comp,
-        "e2e": {"value": round(world * GEMM_FLOP / (e2e_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(d["X"].numel() * 2 + d["W"].numel() * 2),
-                "d2h_bytes_per_step": int(M * N * 2), "ms_per_step": round(e2e_max, 4),
-                "how": "fp4.quantize / fp4.gemm on inputs copied from pinned host memory each step, the whole "
-                       "bf16 result copied back; two buffer sets on 3 streams overlap the copies of "
+                   "parallelism": "independent layer per GPU" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "components": {"per_call": table},
+        "e2e": {"value": round(world * layer.flop / (e2e_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_max, 3),
+                "how": "fp4.quantize / fp4.gemm on the layer's inputs copied from pinned host memory every step, "
+                       "the 12 GEMM outputs copied back; two buffer sets on 3 streams overlap the copies of "
                        "neighbouring steps with each other and with compute"},
-        "gpu_launches": w.launches_per_step * args.steps,
+        "gpu_launches": layer.launches * args.steps,
         "clocks": clocks.summary(),
         "device_status": fp4.fp4_status_string(status),
     }
-    return line
+    return line, layer
 
 
-# ------------------------------------------------------------------------ every config
+# ------------------------------------------------------------------------ other workloads
 
-def _median_ms(fn, flush, reps):
-    """Median CUDA-event time of fn() over reps runs, L2 flushed before each."""
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    fn()
-    ts = []
-    for _ in range(reps):
-        flush()
-        e0.record()
-        fn()
-        e1.record()
-        torch.cuda.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    return statistics.median(ts)
+CONFIG_NAMES = ("fprop", "ufp4", "tiny", "wgrad", "dgrad_db")
 
 
-def _qbytes(x, fmt, db):
-    """Algorithmic bytes of one quantize call: read once, codes + scales (+ outer) written."""
-    n = x.numel()
-    blk = 32 if fmt == 0 else 16
-    return n * x.element_size() + n / 2 + n / blk + (n / 128 * 4 if db else 0)
-
-
-CONFIG_NAMES = ("tiny", "wgrad", "dgrad_db", "layer")
-
-
-def measure_configs(fp4, device, peaks, reps=10, only=CONFIG_NAMES):
-    """Per-kernel timings of every workload (or of those named in `only`):
-    quantize GB/s and GEMM TFLOP/s with their fractions of the measured HBM
-    and derived FP4 peaks."""
+def measure_configs(fp4, device, peaks, layer=None, reps=10, only=CONFIG_NAMES):
+    """Per-kernel timings of the other workloads: quantize GB/s and GEMM TFLOP/s
+    with their fractions of the measured HBM and derived FP4 peaks."""
     flush = L2Flush(device)
     fp4_peak = peaks["bf16"] * 4.0
     out = {}
@@ -382,9 +519,10 @@ def measure_configs(fp4, device, peaks, reps=10, only=CONFIG_NAMES):
         q = fp4.alloc_qtensor(R if axis else C, C if axis else R, fmt, db, device)
         ws = torch.empty(256, dtype=torch.uint8, device=device)
         ms = _median_ms(lambda: fp4.quantize(x, out=q, workspace=ws, **kw), flush, reps)
-        gb = _qbytes(x, fmt, db) + (x.numel() * x.element_size() if (fmt != 0 and not db) else 0)
+        two = fmt != 0 and not db
+        gb = qbytes(x.numel(), x.element_size(), fmt, db, reads=2 if two else 1)
         return q, {"ms": ms, "gbs": gb / (ms * 1e6), "frac_hbm": gb / (ms * 1e6) / peaks["hbm"],
-                   "bytes": "2 reads (amax pass + quantize)" if (fmt != 0 and not db) else "1 read"}
+                   "bytes": "2 reads (amax pass + quantize)" if two else "1 read"}
 
     def gemm_entry(qa, qb, out_dtype):
         M, N, K = qa["lines"], qb["lines"], qa["K"]
@@ -395,6 +533,24 @@ def measure_configs(fp4, device, peaks, reps=10, only=CONFIG_NAMES):
 
     NV, MX, UF = fp4.FP4_NVFP4, fp4.FP4_MXFP4, fp4.FP4_UFP4
     BF, F32 = fp4.FP4_OUT_BF16, fp4.FP4_OUT_F32
+
+    if "fprop" in only:
+        out["nvfp4_fprop_qkv_8192x6144x4096"] = fprop_component(fp4, device, flush, peaks, reps)
+
+    if "ufp4" in only and layer is not None:
+        # the UFP4 quantizer (levels k * s, k in [-7, 7]) on the layer's operands
+        uf = {}
+        tot_ms = tot_b = 0.0
+        for lin in layer.linears:
+            for role, c in enumerate(lin["calls"]):
+                x = lin["t"][c["x"]]
+                _, e = quant_entry(x, fmt=UF, rounding=c["rounding"], rotation=fp4.FP4_ROT_H16, axis=c["axis"],
+                                   seed=0, tensor_id=c["tensor_id"])
+                uf.setdefault(lin["name"], {})[c["name"]] = e
+                tot_ms += e["ms"]
+                tot_b += e["gbs"] * e["ms"] * 1e6
+        out["ufp4_layer_quantize"] = {"calls": uf, "total_ms": tot_ms, "gbs": tot_b / (tot_ms * 1e6),
+                                      "frac_hbm": tot_b / (tot_ms * 1e6) / peaks["hbm"]}
 
     if "tiny" in only:
         d = workloads.tiny_mxfp4()
@@ -433,112 +589,131 @@ def measure_configs(fp4, device, peaks, reps=10, only=CONFIG_NAMES):
                                       "bytes": "FP4 source read + FP4 result written"}
         out["nvfp4_dgrad_down_db_8192x14336x4096"] = entry
         del dY, Wd, qa, qb, fwd, back
-    if "layer" not in only:
-        return out
-
-    # the decoder layer: Fprop, Dgrad, Wgrad of each linear in NVFP4 with H16
-    # (SR on the Wgrad operands), then the UFP4 quantizer on the same operands
-    layer = {"quantize_nvfp4_ms": 0.0, "quantize_ufp4_ms": 0.0, "quantize_bytes": 0.0, "gemm_ms": 0.0,
-             "gemm_flop": 0.0, "linears": {}}
-    for name, _, _, _ in workloads.LAYER_LINEARS:
-        d = workloads.layer_linear(name)
-        X, W, dY = d["X"].to(device), d["W"].to(device), d["dY"].to(device)
-        H16, SR, RT = fp4.FP4_ROT_H16, fp4.FP4_SR, fp4.FP4_RTNE
-        ops = {"X_ax1": (X, 1, RT), "W_ax1": (W, 1, RT), "dY_ax1": (dY, 1, RT), "W_ax0": (W, 0, RT),
-               "dY_ax0": (dY, 0, SR), "X_ax0": (X, 0, SR)}
-        lin = {}
-        qs = {}
-        for role, (t, axis, rnd) in ops.items():
-            qs[role], e = quant_entry(t, fmt=NV, rounding=rnd, rotation=H16, axis=axis, seed=0, tensor_id=len(qs))
-            _, u = quant_entry(t, fmt=UF, rounding=rnd, rotation=H16, axis=axis, seed=0, tensor_id=len(qs))
-            lin["nv_" + role], lin["uf_" + role] = e, u
-            layer["quantize_nvfp4_ms"] += e["ms"]
-            layer["quantize_ufp4_ms"] += u["ms"]
-            layer["quantize_bytes"] += e["gbs"] * e["ms"] * 1e6
-        for gname, (a_, b_, od) in {"fprop": ("X_ax1", "W_ax1", BF), "dgrad": ("dY_ax1", "W_ax0", BF),
-                                    "wgrad": ("dY_ax0", "X_ax0", F32)}.items():
-            g = gemm_entry(qs[a_], qs[b_], od)
-            lin[gname] = g
-            layer["gemm_ms"] += g["ms"]
-            layer["gemm_flop"] += 2.0 * g["shape"][0] * g["shape"][1] * g["shape"][2]
-        layer["linears"][name] = lin
-        del X, W, dY, qs
-        torch.cuda.empty_cache()
-    layer["gemm_tflops"] = layer["gemm_flop"] / (layer["gemm_ms"] * 1e-3) / 1e12
-    layer["gemm_frac_fp4"] = layer["gemm_tflops"] / fp4_peak
-    layer["quantize_nvfp4_gbs"] = layer["quantize_bytes"] / (layer["quantize_nvfp4_ms"] * 1e6)
-    layer["quantize_nvfp4_frac_hbm"] = layer["quantize_nvfp4_gbs"] / peaks["hbm"]
-    out["llama8b_layer_linears_t8192"] = layer
+    torch.cuda.empty_cache()
     return out
 
 
-# ------------------------------------------------------------------------ oracle arm
+# ------------------------------------------------------------------------ oracle (CPU) arm
 
-def oracle_slab_time(d, rows):
-    """Oracle time of the step restricted to `rows` rows of X and of W,
-    extrapolated to the whole workload (seconds), and the threads it used."""
+ORACLE_SLAB = 128
+
+
+def oracle_layer_sample(host):
+    """The oracle, as it stands, on a fixed sample of the layer step, and the
+    step time extrapolated from it.
+
+    Per linear: for each of the six NVFP4 + H16 operands, the rotated amax of
+    its first 128 lines and the quantization of those lines given that amax
+    (each extrapolated by lines / 128); for each GEMM, the dequantization of
+    the two 128-line slabs and the oracle GEMM of the slabs (float64 product
+    and bound), the dequantization extrapolated by (M + N) / 256 and the
+    product by M N / 128^2.  Returns the extrapolated quantize and GEMM times
+    (s), the wall time spent, and the work they stand for."""
     import oracle
-    X = workloads.bf16_bits(d["X"][:rows])
-    W = workloads.bf16_bits(d["W"][:rows])
-    t0 = time.perf_counter()
-    ax = oracle.tensor_amax(X, 1, oracle.ROT_H16)
-    t1 = time.perf_counter()
-    qx = oracle.quantize(X, oracle.NVFP4, rotation=oracle.ROT_H16, amax=ax)
-    t2 = time.perf_counter()
-    aw = oracle.tensor_amax(W, 1, oracle.ROT_H16)
-    t3 = time.perf_counter()
-    qw = oracle.quantize(W, oracle.NVFP4, rotation=oracle.ROT_H16, amax=aw)
-    t4 = time.perf_counter()
-    oracle.gemm(qx, qw)
-    t5 = time.perf_counter()
-    full = ((t2 - t0) * M / rows + (t4 - t2) * N / rows + (t5 - t4) * (M * N) / (rows * rows))
-    return full, oracle.default_threads()
+    t_amax = t_q = t_dq = t_mm = 0.0
+    quant_bytes = flop = 0.0
+    wall0 = time.perf_counter()
+    for index, d in enumerate(host):
+        qs = []
+        for role, (tn, axis, sr) in enumerate(OPERANDS):
+            x = d[tn]
+            R, C = x.shape
+            L = R if axis == 1 else C
+            slab = x[:ORACLE_SLAB] if axis == 1 else np.ascontiguousarray(x[:, :ORACLE_SLAB])
+            t0 = time.perf_counter()
+            a = oracle.tensor_amax(slab, axis, oracle.ROT_H16)
+            t1 = time.perf_counter()
+            q = oracle.quantize(x, oracle.NVFP4, rounding=oracle.SR if sr else oracle.RTNE, rotation=oracle.ROT_H16,
+                                axis=axis, seed=0, tensor_id=workloads.layer_tensor_id(index, role), amax=a,
+                                lines=np.arange(ORACLE_SLAB))
+            t2 = time.perf_counter()
+            t_amax += (t1 - t0) * L / ORACLE_SLAB
+            t_q += (t2 - t1) * L / ORACLE_SLAB
+            quant_bytes += qbytes(R * C, 2, 1, reads=2)
+            qs.append((q, L))
+        for _, ra, rb, _ in GEMMS:
+            (qa, M), (qb, N) = qs[ra], qs[rb]
+            K = qa["K"]
+            t0 = time.perf_counter()
+            oracle.dequantize(qa)
+            oracle.dequantize(qb)
+            t1 = time.perf_counter()
+            oracle.gemm(qa, qb)
+            t2 = time.perf_counter()
+            dq = t1 - t0
+            t_dq += dq * (M + N) / (2 * ORACLE_SLAB)
+            t_mm += max(t2 - t1 - dq, 0.0) * (M * N) / (ORACLE_SLAB * ORACLE_SLAB)
+            flop += 2.0 * M * N * K
+    wall = time.perf_counter() - wall0
+    return dict(t_quant=t_amax + t_q, t_gemm=t_dq + t_mm, wall=wall, quant_bytes=quant_bytes, flop=flop,
+                t_amax=t_amax, t_q=t_q, t_dq=t_dq, t_mm=t_mm)
 
 
-def cpu_baseline(d, target_s=10.0):
-    rows = 64
-    t, cores = oracle_slab_time(d, rows)
-    # grow the slab towards ~target_s of CPU work
-    spent = t * rows / M
-    if spent < target_s / 4:
-        rows = int(min(1024, rows * target_s / 2 / max(spent, 1e-3)))
-        rows = max(64, rows - rows % 16)
-        t, cores = oracle_slab_time(d, rows)
-    value = GEMM_FLOP / t / 1e12
-    return {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": "%d rows of X and of W: amax + quantize (NVFP4, H16) and the float64 GEMM of "
-                      "the %dx%d slab, each part extrapolated to the full 8192x6144x4096 step" % (rows, rows, rows)}
+SAMPLE_DESC = ("per linear of the layer: the rotated amax and the NVFP4 + H16 quantization of the first %d lines "
+               "of each of the 6 operands, and the oracle GEMM (exact dequantization, float64 product and bound) "
+               "of %d x %d line slabs of each of the 3 GEMMs; extrapolated to the full layer step "
+               "(quantize by lines, dequantization by M + N, product by M N)" % (ORACLE_SLAB, ORACLE_SLAB,
+                                                                                 ORACLE_SLAB))
+
+
+def oracle_baseline_entry(res, ms_per_sample=None):
+    import oracle
+    t_full = res["t_quant"] + res["t_gemm"]
+    e = {"value": res["flop"] / t_full / 1e12, "unit": "TFLOP/s", "cores": oracle.default_threads(),
+         "kind": "oracle", "sample": SAMPLE_DESC, "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+         "extrapolated_step_s": t_full,
+         "quantize_gbs": res["quant_bytes"] / res["t_quant"] / 1e9,
+         "gemm_gflops": res["flop"] / res["t_gemm"] / 1e9,
+         "quantize_bytes_are": "2 reads of the bf16 input (amax pass + quantize) + codes and scales written"}
+    if ms_per_sample is not None:
+        e["sample_wall_ms"] = ms_per_sample
+    return e
+
+
+def cpu_baseline(host, reps=3):
+    """The oracle sample `reps` times; the median extrapolated step."""
+    runs = [oracle_layer_sample(host) for _ in range(reps)]
+    runs.sort(key=lambda r: r["t_quant"] + r["t_gemm"])
+    res = runs[len(runs) // 2]
+    return oracle_baseline_entry(res, statistics.median(r["wall"] for r in runs) * 1e3)
+
+
+def layer_host_data(seed=0):
+    return [workloads.layer_linear(name, seed=seed) for name, _, _, _ in workloads.LAYER_LINEARS]
+
+
+def host_bits(host):
+    return [{k: workloads.bf16_bits(v) for k, v in d.items()} for d in host]
 
 
 def run_reference(args):
-    """The oracle, as it stands, timed on the host cores on a bounded sample."""
-    d = workloads.nvfp4_fprop_qkv(seed=0)
-    budget_s = 120.0                              # wall time of the whole run
-    steps = args.steps + args.warmup
-    # calibrate on a 64-row slab, then take the largest slab (a multiple of 16
-    # rows, at most 1024) whose steps fit the budget: small slabs are
-    # dominated by fixed costs and understate the oracle's rate
-    t0 = time.perf_counter()
-    oracle_slab_time(d, 64)
-    wall64 = time.perf_counter() - t0
-    rows = int(64 * budget_s / (steps * max(wall64, 1e-4)))
-    rows = max(16, min(1024, rows - rows % 16))
-    times = []
+    """The oracle, as it stands, timed on the host cores: each step is the fixed
+    sample of the layer step (oracle_layer_sample); `value` is the step's GEMM
+    FLOP over the step time extrapolated from the sample, `ms_per_step` the
+    measured wall time of one sampled step."""
+    bits = host_bits(layer_host_data(seed=0))
+    runs = []
     for i in range(args.warmup + args.steps):
-        t, cores = oracle_slab_time(d, rows)
+        r = oracle_layer_sample(bits)
         if i >= args.warmup:
-            times.append(t)
-    ms = statistics.mean(times) * 1e3
-    value = GEMM_FLOP / (ms * 1e-3) / 1e12
+            runs.append(r)
+    wall_ms = statistics.mean(r["wall"] for r in runs) * 1e3
+    runs.sort(key=lambda r: r["t_quant"] + r["t_gemm"])
+    res = runs[len(runs) // 2]
+    base = oracle_baseline_entry(res, wall_ms)
+    value = base["value"]
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizer, f64 GEMM (CPU oracle)",
-        "data": "synthetic (same seeded workload)",
-        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "format": "NVFP4", "rotation": "H16",
-                   "rounding": "RTNE", "out": "f64"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": "per step: %d rows of X and W through the whole step, extrapolated" % rows},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall_ms, 3),
+        "ms_per_step_is": "measured wall time of one sampled oracle step (not the full layer step)",
+        "extrapolated_full_step_ms": round(base["extrapolated_step_s"] * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 quantizer, f64 GEMM (CPU oracle)", "data": "synthetic (same seeded workload)",
+        "config": {"workload": WORKLOAD, "tokens": T,
+                   "linears": {n: [d_in, d_out] for n, d_in, d_out, _ in workloads.LAYER_LINEARS},
+                   "format": "NVFP4", "rotation": "H16 on all three GEMMs",
+                   "rounding": "RTNE; SR on the Wgrad operands", "out": "f64"},
+        "cpu_baseline": base,
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -546,13 +721,13 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["fp4", "reference"], default="fp4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel table")
     ap.add_argument("--graph", action="store_true",
-                    help="time the step replayed as one CUDA graph (measured equal to eager launches)")
+                    help="time the step replayed as one CUDA graph")
     ap.add_argument("--configs", default=",".join(CONFIG_NAMES),
                     help="comma-separated workloads of the per-config table: " + ", ".join(CONFIG_NAMES))
     args = ap.parse_args()
@@ -573,7 +748,8 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
-    line = run_gpu(args, rank, world, device)
+    host = layer_host_data(seed=rank)
+    line, layer = run_gpu(args, rank, world, device, host=host)
     if rank == 0:
         if world == 1 and not args.no_configs:
             from fp4_block_scaled_h16_b200 import fp4 as _fp4
@@ -581,9 +757,11 @@ def main():
             unknown = [c for c in only if c not in CONFIG_NAMES]
             if unknown:
                 raise SystemExit("unknown --configs entries: %s" % ", ".join(unknown))
-            line["configs"] = measure_configs(_fp4, device, measured_peaks(), only=only)
+            line["components"].update(measure_configs(_fp4, device, measured_peaks(), layer=layer, only=only))
+        del layer
+        torch.cuda.empty_cache()
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(workloads.nvfp4_fprop_qkv(seed=0))
+            line["cpu_baseline"] = cpu_baseline(host_bits(host))
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

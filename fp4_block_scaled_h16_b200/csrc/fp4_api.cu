@@ -180,6 +180,25 @@ fp4_status_t fp4_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int6
     return FP4_OK;
 }
 
+fp4_status_t fp4_rotate(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                        fp4_rotation_t rotation, int axis, uint64_t seed, void* y, int64_t ldy, void* stream) {
+    fp4_status_t st = check_input(x, in_dtype, rows, cols, ld, rotation, axis);
+    if (st != FP4_OK) return st;
+    if (axis != 1) return FP4_ERR_UNSUPPORTED;
+    if (rotation == FP4_ROT_NONE) return FP4_ERR_INVALID_ARG;
+    if (ldy < cols) return FP4_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return FP4_OK;
+    const int64_t es = in_dtype == FP4_IN_BF16 ? 2 : 4;
+    if (!y) return FP4_ERR_INVALID_ARG;
+    if (!aligned16(y) || (ldy * es) % 16) return FP4_ERR_MISALIGNED;
+    int dev;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    if (launch_rotate_rows(x, y, in_dtype == FP4_IN_BF16, rows, cols, ld, ldy, rot_size(rotation),
+                           sign_mask_of(rotation, seed), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
 fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
                           fp4_format_t format, fp4_rounding_t rounding, fp4_rotation_t rotation, int axis,
                           int double_block, uint64_t seed, uint32_t tensor_id, const float* tensor_amax,

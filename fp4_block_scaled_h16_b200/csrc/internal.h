@@ -51,6 +51,9 @@ cudaError_t launch_amax_cols(const QuantArgs& a, bool bf16, int rot_n, bool sign
 cudaError_t launch_requantize_cols(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db,
                                    cudaStream_t s);
 cudaError_t launch_requant_amax_cols(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s);
+// the rotation alone along the rows (fp4_rotate)
+cudaError_t launch_rotate_rows(const void* x, void* y, bool bf16, int64_t rows, int64_t cols, int64_t ld,
+                               int64_t ldy, int n, uint32_t sign_mask, cudaStream_t s);
 
 // GEMM
 struct GemmArgs {

@@ -33,7 +33,7 @@ FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
 
 EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_quantize",
            "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit",
-           "fp4_quantize_noalloc", "fp4_requantize")
+           "fp4_quantize_noalloc", "fp4_requantize", "fp4_rotate")
 
 _P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_uint32, ctypes.c_size_t)
@@ -48,11 +48,12 @@ _lib.fp4_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _I, _U64
 _lib.fp4_quantize_noalloc.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P]
 _lib.fp4_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P, _P,
                                 _P, _SZ, _P]
+_lib.fp4_rotate.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _P, _I64, _P]
 _lib.fp4_gemm.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P]
 _lib.fp4_last_error.argtypes = [_P]
 _lib.fp4_set_wait_limit.argtypes = [_U32]
 _lib.fp4_set_wait_limit.restype = None
-for _f in ("fp4_amax", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
+for _f in ("fp4_amax", "fp4_rotate", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
            "fp4_quantize_workspace_size"):
     getattr(_lib, _f).restype = _I
 
@@ -107,6 +108,21 @@ def fp4_set_wait_limit(polls: int) -> None:
 def fp4_amax(x, in_dtype, rows, cols, ld, rotation, axis, seed, amax_out, stream=None) -> None:
     _check(_lib.fp4_amax(_ptr(x), in_dtype, rows, cols, ld, rotation, axis, seed, _ptr(amax_out),
                          _stream(stream)), "fp4_amax")
+
+
+def fp4_rotate(x, in_dtype, rows, cols, ld, rotation, axis, seed, y, ldy, stream=None) -> None:
+    _check(_lib.fp4_rotate(_ptr(x), in_dtype, rows, cols, ld, rotation, axis, seed, _ptr(y), ldy,
+                           _stream(stream)), "fp4_rotate")
+
+
+def rotate(x, rotation, seed=0, out=None, stream=None):
+    """The rotation alone along the rows of a 2-D CUDA tensor, in its own dtype (fp4_rotate)."""
+    import torch
+    rows, cols = x.shape
+    ld = x.stride(0) if rows > 1 else cols
+    y = out if out is not None else torch.empty((rows, cols), dtype=x.dtype, device=x.device)
+    fp4_rotate(x, in_dtype_of(x), rows, cols, ld, rotation, 1, seed, y, y.stride(0) if rows > 1 else cols, stream)
+    return y
 
 
 def fp4_quantize(x, in_dtype, rows, cols, ld, fmt, rounding, rotation, axis, double_block, seed,

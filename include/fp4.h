@@ -123,6 +123,25 @@ fp4_status_t fp4_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int6
                       float* amax_out, void* stream);
 
 /*
+ * fp4_rotate -- the rotation of fp4_quantize's step 2 alone, as a separate
+ * pass: y = c_n * H_n * (d . x) on every aligned n-block of each row, in
+ * binary32 with the same operation order, stored in the input's type (bf16:
+ * rounded to nearest even).  "Ripensare il Bias di Shrinkage nel Pretraining
+ * di LLM in FP4", Efficienza: the pages time a separate rotation kernel
+ * followed by the quantizer against the fused quantizer; this call is that
+ * separate kernel.
+ *
+ *   x, in_dtype, rows, cols, ld   input [rows, ld] row-major (as fp4_quantize)
+ *   rotation        FP4_ROT_H16 / H32 / RH16 / RH32 (not NONE); n divides cols
+ *   axis            must be 1 (rows); any other value returns FP4_ERR_UNSUPPORTED
+ *   seed            the random signs of RH16 / RH32
+ *   y, ldy          device, [rows, ldy] of the input's type, ldy >= cols,
+ *                   16-byte aligned; may not overlap x
+ */
+fp4_status_t fp4_rotate(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                        fp4_rotation_t rotation, int axis, uint64_t seed, void* y, int64_t ldy, void* stream);
+
+/*
  * fp4_quantize -- fused rotate / amax / scale / round / pack of one tensor.
  *
  * Steps, on every line of K elements along `axis`:

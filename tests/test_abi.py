@@ -130,11 +130,30 @@ def test_requantize_host_validation(kw, status):
     assert rq(**kw) == status
 
 
+@pytest.mark.skipif(torch.cuda.is_available(), reason="an empty call writes tensor_scale: the fake address "
+                    "must never reach a GPU")
 def test_empty_requantize_is_a_no_op_without_gpu_work():
-    assert rq(lines=0, sc=None, ss=None, codes=None, scales=None, ws=None) in (0, fp4.FP4_ERR_NO_DEVICE)
+    assert rq(lines=0, sc=None, ss=None, codes=None, scales=None, ws=None) == fp4.FP4_ERR_NO_DEVICE
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
 def test_valid_call_without_gpu_reports_no_device():
     assert q() == fp4.FP4_ERR_NO_DEVICE
     assert g() == fp4.FP4_ERR_NO_DEVICE
+
+
+def rot(**kw):
+    a = dict(x=ADDR, dt=fp4.FP4_IN_BF16, rows=64, cols=256, ld=256, rotation=fp4.FP4_ROT_H16, axis=1, seed=0,
+             y=ADDR, ldy=256)
+    a.update(kw)
+    return fp4._lib.fp4_rotate(a["x"], a["dt"], a["rows"], a["cols"], a["ld"], a["rotation"], a["axis"], a["seed"],
+                               a["y"], a["ldy"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dt=3), 1), (dict(rotation=0), 1), (dict(rotation=9), 1), (dict(ldy=128), 1), (dict(y=None), 1),
+    (dict(axis=0), 8), (dict(cols=248, ld=256), 2), (dict(rotation=fp4.FP4_ROT_H32, cols=240, ld=256), 2),
+    (dict(y=ADDR + 8), 3), (dict(ldy=260), 3), (dict(x=ADDR + 2), 3),
+])
+def test_rotate_host_validation(kw, status):
+    assert rot(**kw) == status
