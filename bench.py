@@ -139,10 +139,10 @@ def qbytes(numel, elem_bytes, fmt, db=False, reads=1):
 
 
 def quantize_kernels(axis, internal_amax):
-    """Kernels one fp4_quantize call launches: the row axis runs the amax and
-    quantize passes as one cooperative kernel; axis 0 runs an amax kernel then
-    the quantize kernel; with a given amax (or MXFP4 / double block) one."""
-    return 2 if (internal_amax and axis == 0) else 1
+    """Kernels one fp4_quantize call launches: one on either axis (with an
+    internal tensor amax, the amax and quantize passes run as one cooperative
+    kernel)."""
+    return 1
 
 
 # ------------------------------------------------------------------------ GPU arm

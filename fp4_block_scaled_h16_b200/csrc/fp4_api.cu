@@ -259,12 +259,10 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
         a.amax_out = static_cast<unsigned int*>(workspace);
         a.grid_count = static_cast<unsigned int*>(workspace) + 1;
         a.amax_in = static_cast<const float*>(workspace);
-        if (axis == 1) {
-            // one launch: amax pass, grid barrier, quantize pass
-            if (launch_quantize_fused(a, bf16, format, rounding == FP4_SR, rn, s) != cudaSuccess) return FP4_ERR_CUDA;
-            return FP4_OK;
-        }
-        if (launch_amax(a, bf16, rn, axis, s) != cudaSuccess) return FP4_ERR_CUDA;
+        // one launch on either axis: amax pass, grid barrier, quantize pass
+        if (launch_quantize_fused(a, bf16, format, rounding == FP4_SR, rn, axis, s) != cudaSuccess)
+            return FP4_ERR_CUDA;
+        return FP4_OK;
     } else {
         a.amax_in = tensor_amax;
     }

@@ -41,12 +41,19 @@ struct QuantArgs {
 cudaError_t launch_quantize(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, bool db, int axis,
                             cudaStream_t s);
 cudaError_t launch_amax(QuantArgs a, bool bf16, int rot_n, int axis, cudaStream_t s);
-// NVFP4 / UFP4, row axis: amax pass, grid barrier and quantize pass in one
+// NVFP4 / UFP4, either axis: amax pass, grid barrier and quantize pass in one
 // cooperative launch; a.amax_out / a.grid_count point at zeroed words
-cudaError_t launch_quantize_fused(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, cudaStream_t s);
-cudaError_t launch_quantize_cols(const QuantArgs& a, bool bf16, int fmt, bool sr, int rot_n, bool signs,
-                                 bool db, cudaStream_t s);
-cudaError_t launch_amax_cols(const QuantArgs& a, bool bf16, int rot_n, bool signs, cudaStream_t s);
+cudaError_t launch_quantize_fused(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, int axis, cudaStream_t s);
+// the same for axis 0 (quant_cols.cuh), per input type
+template <bool BF16>
+cudaError_t launch_cols_quantize(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db, cudaStream_t s);
+template <bool BF16>
+cudaError_t launch_cols_amax(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s);
+template <bool BF16>
+cudaError_t launch_cols_fused(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, cudaStream_t s);
+// 2-D TMA map over a [rows, cols] input of row pitch ld, box 64 columns x 128
+// rows, no swizzle, zeros past the edges
+bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld);
 // the same two along axis 0 of the dequantized source (a.src_*)
 cudaError_t launch_requantize_cols(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db,
                                    cudaStream_t s);

@@ -26,6 +26,12 @@ namespace fp4 {
 extern template cudaError_t launch_rows_quantize<false>(const QuantArgs&, int, bool, int, bool, bool, cudaStream_t);
 extern template cudaError_t launch_rows_amax<false>(const QuantArgs&, int, bool, cudaStream_t);
 extern template cudaError_t launch_rows_fused<false>(const QuantArgs&, int, bool, int, bool, cudaStream_t);
+extern template cudaError_t launch_cols_quantize<true>(const QuantArgs&, int, bool, int, bool, bool, cudaStream_t);
+extern template cudaError_t launch_cols_quantize<false>(const QuantArgs&, int, bool, int, bool, bool, cudaStream_t);
+extern template cudaError_t launch_cols_amax<true>(const QuantArgs&, int, bool, cudaStream_t);
+extern template cudaError_t launch_cols_amax<false>(const QuantArgs&, int, bool, cudaStream_t);
+extern template cudaError_t launch_cols_fused<true>(const QuantArgs&, int, bool, int, bool, cudaStream_t);
+extern template cudaError_t launch_cols_fused<false>(const QuantArgs&, int, bool, int, bool, cudaStream_t);
 
 namespace {
 
@@ -47,14 +53,19 @@ int unit_of(int fmt, int rot_n, int64_t K) {
 cudaError_t launch_quantize(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, bool db, int axis,
                             cudaStream_t s) {
     const bool signs = a.sign_mask != 0u;
-    if (axis == 0) return launch_quantize_cols(a, bf16, fmt, sr, rot_n, signs, db, s);
+    if (axis == 0)
+        return bf16 ? launch_cols_quantize<true>(a, fmt, sr, rot_n, signs, db, s)
+                    : launch_cols_quantize<false>(a, fmt, sr, rot_n, signs, db, s);
     set_divisor(a, (uint32_t)(a.K / unit_of(fmt, rot_n, a.K)));
     return bf16 ? launch_rows_quantize<true>(a, fmt, sr, rot_n, signs, db, s)
                 : launch_rows_quantize<false>(a, fmt, sr, rot_n, signs, db, s);
 }
 
-cudaError_t launch_quantize_fused(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, cudaStream_t s) {
+cudaError_t launch_quantize_fused(QuantArgs a, bool bf16, int fmt, bool sr, int rot_n, int axis, cudaStream_t s) {
     const bool signs = a.sign_mask != 0u;
+    if (axis == 0)
+        return bf16 ? launch_cols_fused<true>(a, fmt, sr, rot_n, signs, s)
+                    : launch_cols_fused<false>(a, fmt, sr, rot_n, signs, s);
     set_divisor(a, (uint32_t)(a.K / unit_of(fmt, rot_n, a.K)));
     return bf16 ? launch_rows_fused<true>(a, fmt, sr, rot_n, signs, s)
                 : launch_rows_fused<false>(a, fmt, sr, rot_n, signs, s);
@@ -62,7 +73,7 @@ cudaError_t launch_quantize_fused(QuantArgs a, bool bf16, int fmt, bool sr, int 
 
 cudaError_t launch_amax(QuantArgs a, bool bf16, int rot_n, int axis, cudaStream_t s) {
     const bool signs = a.sign_mask != 0u;
-    if (axis == 0) return launch_amax_cols(a, bf16, rot_n, signs, s);
+    if (axis == 0) return bf16 ? launch_cols_amax<true>(a, rot_n, signs, s) : launch_cols_amax<false>(a, rot_n, signs, s);
     set_divisor(a, (uint32_t)(a.K / unit_of(NVFP4, rot_n, a.K)));
     return bf16 ? launch_rows_amax<true>(a, rot_n, signs, s) : launch_rows_amax<false>(a, rot_n, signs, s);
 }

@@ -1,7 +1,9 @@
-// quantize_cols.cu -- the transposed-axis (axis = 0) quantizer: blocks run down
-// the columns of the row-major input and the output lines are its columns, as
-// the Dgrad / Wgrad operands need ("TetraJet-v2" 2.A: 1x16 groups re-aligned
-// for the transposed weight).  Same arithmetic as the row-axis kernel.
+// requantize_cols.cu -- fp4_requantize's kernel: the transposed-axis (axis = 0)
+// quantizer reading its tile from an already quantized tensor, X^ = the exact
+// dequantized values rounded once to binary32 ("TetraJet-v2" 2.A: the backward
+// pass estimates with X^, and the 1x16 groups are re-aligned for the
+// transposed weight).  Blocks run down the columns of X^ and the output lines
+// are its columns; same arithmetic as the other quantizer kernels.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -32,9 +34,11 @@ __device__ __forceinline__ __half2 e2m1x2_to_h2(uint32_t byte) {
 }
 
 // FP4SRC: the tile is the dequantized source X^ (fp4_requantize) instead of x
+// (only FP4SRC = true is instantiated; bf16 / f32 input has its own kernel in
+// quant_cols.cuh)
 template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY, bool FP4SRC = false>
 __global__ void __launch_bounds__(T0_THREADS, 4)
-quant_cols_kernel(const QuantArgs a) {
+requant_cols_kernel(const QuantArgs a) {
     __shared__ __align__(16) float tile[T0_ROWS][T0_COLS + 4];
     __shared__ float chunk_max[4][T0_COLS];
     const int64_t R = a.rows, C = a.cols;
@@ -264,7 +268,7 @@ namespace {
 template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, bool AMAX_ONLY, bool FP4SRC>
 cudaError_t launch_cols(const QuantArgs& a, cudaStream_t s) {
     dim3 grid((unsigned)((a.cols + T0_COLS - 1) / T0_COLS), (unsigned)((a.rows + T0_ROWS - 1) / T0_ROWS));
-    quant_cols_kernel<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY, FP4SRC><<<grid, T0_THREADS, 0, s>>>(a);
+    requant_cols_kernel<BF16, FMT, SR, ROT, SIGNS, DB, AMAX_ONLY, FP4SRC><<<grid, T0_THREADS, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -290,17 +294,6 @@ cudaError_t cols_by_fmt(const QuantArgs& a, int fmt, bool sr, int rot_n, bool si
 }
 
 }  // namespace
-
-cudaError_t launch_quantize_cols(const QuantArgs& a, bool bf16, int fmt, bool sr, int rot_n, bool signs,
-                                 bool db, cudaStream_t s) {
-    return bf16 ? cols_by_fmt<true>(a, fmt, sr, rot_n, signs, db, s)
-                : cols_by_fmt<false>(a, fmt, sr, rot_n, signs, db, s);
-}
-
-cudaError_t launch_amax_cols(const QuantArgs& a, bool bf16, int rot_n, bool signs, cudaStream_t s) {
-    return bf16 ? cols_by_rot<true, NVFP4, false, false, true>(a, rot_n, signs, s)
-                : cols_by_rot<false, NVFP4, false, false, true>(a, rot_n, signs, s);
-}
 
 cudaError_t launch_requantize_cols(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db,
                                    cudaStream_t s) {
