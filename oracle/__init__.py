@@ -87,6 +87,9 @@ def lib():
         L.orc_quantize_lines.argtypes = [P, i32, i64, i64, i64, i32, i32, i32, i32, i32,
                                          u64, u32, f32, i64, i64, P, P, P]
         L.orc_dequantize.argtypes = [P, P, P, f32, i64, i64, i32, i32, P]
+        L.orc_pairwise_sum.argtypes = [P, i64]
+        L.orc_pairwise_sum.restype = ctypes.c_double
+        L.orc_mxnorm_rho.argtypes = [P, i32, i64, i64, i64, i32, i32, ctypes.c_double, i64, i64, P, P]
         _lib = L
     return _lib
 
@@ -302,3 +305,77 @@ def gemm(qa: dict, qb: dict):
     a = dequantize(qa)
     b = dequantize(qb)
     return a @ b.T, np.abs(a) @ np.abs(b).T
+
+
+# --------------------------------------------------------------------------- MXNorm
+
+def pairwise_sum(a) -> float:
+    """binary64 sum of a in index order, pairwise (halves split at the largest
+    power of two below the length): the order MXNorm's block statistic uses."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    return lib().orc_pairwise_sum(_ptr(a), len(a))
+
+
+def mxnorm_rho(x: np.ndarray, block: int, p: int, c: float, C: int | None = None,
+               threads: int | None = None):
+    """Per-row inverse-RMS estimate rho_t = c * ((1/K) sum_k m_tk^p)^(-1/p) from
+    the block maxima m_tk ("MXNorm: Reusing MXFP block scales...", 2.
+    Metodologia), as binary32, and each row's max |x|."""
+    x = np.ascontiguousarray(x)
+    dt = _as_input(x)
+    R, ld = x.shape
+    C = ld if C is None else C
+    rho = np.zeros(R, np.float32)
+    rmax = np.zeros(R, np.float32)
+    threads = threads or default_threads()
+    L = lib()
+
+    def run(rng):
+        a, b = rng
+        rc = L.orc_mxnorm_rho(_ptr(x), dt, R, C, ld, block, p, float(c), a, b, _ptr(rho[a:b]), _ptr(rmax[a:b]))
+        if rc:
+            raise ValueError("oracle rejected the MXNorm shape or p (code %d)" % rc)
+
+    parts = _chunks(0, R, threads)
+    if parts:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(run, parts))
+    return rho, rmax
+
+
+def widen(x: np.ndarray) -> np.ndarray:
+    """binary32 values of an oracle input (float32, or bf16 bit patterns)."""
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32)
+    return np.asarray(x, dtype=np.float32)
+
+
+def mxnorm(x: np.ndarray, fmt: int, p: int, c: float, rounding: int = RTNE, seed: int = 0,
+           tensor_id: int = 0, C: int | None = None, lines=None) -> dict:
+    """MXNorm fused with the cast: rho per row from the format's block maxima
+    (32 for MXFP4, 16 for NVFP4 / UFP4), y = RN32(x * rho), and y quantized
+    along the rows without rotation (the gain is folded into the next
+    layer's weight, as the page does).  Returns the quantized dict of
+    `quantize` with `rho` and `y` added."""
+    x = np.ascontiguousarray(x)
+    R, ld = x.shape
+    C = ld if C is None else C
+    block = 32 if fmt == MXFP4 else 16
+    rho, _ = mxnorm_rho(x, block, p, c, C=C)
+    y = (widen(x)[:, :C] * rho[:, None]).astype(np.float32)     # one binary32 rounding per element
+    q = quantize(np.ascontiguousarray(y), fmt, rounding=rounding, rotation=ROT_NONE, axis=1, seed=seed,
+                 tensor_id=tensor_id, lines=lines)
+    q["rho"] = rho
+    q["y"] = y
+    return q
+
+
+def mxnorm_constant(p: int, block: int) -> float:
+    """c(p, B) for rows of i.i.d. Gaussian values: E[M^p]^(1/p) with M the
+    maximum of B independent |N(0, 1)|, so that rho_t times the row's RMS
+    tends to 1 (the page obtains c by Monte Carlo; here by quadrature of
+    E[M^p] = int_0^inf p m^(p-1) (1 - erf(m / sqrt 2)^B) dm)."""
+    from scipy import integrate, special
+    f = lambda m: p * m ** (p - 1) * (1.0 - special.erf(m / np.sqrt(2.0)) ** block)
+    val, _ = integrate.quad(f, 0.0, np.inf, epsabs=1e-13, epsrel=1e-12, limit=200)
+    return float(val ** (1.0 / p))

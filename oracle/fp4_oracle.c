@@ -413,3 +413,67 @@ int orc_dequantize(const uint8_t* codes, const uint8_t* scales, const float* out
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXNorm ("MXNorm: Reusing MXFP block scales for efficient tensor            */
+/* normalisation", 2. Metodologia): the inverse RMS of a row t is estimated   */
+/* from the absolute maxima m_tk of its K blocks of B elements,               */
+/*     rho_t = c(p, B) * ((1/K) sum_k m_tk^p)^(-1/p),                          */
+/* and the normalised row y = x * rho_t is what the MX cast quantizes.        */
+/* Readings (the pages give the formula only): m_tk in binary32 (exact); the  */
+/* sum in binary64, pairwise in block order (a range's sum is the sum of its  */
+/* two halves, split at the largest power of two below its length); the      */
+/* mean, the square root (p = 2) and c / g in binary64, each correctly        */
+/* rounded, then one rounding to binary32, saturating at the largest finite   */
+/* binary32; an all-zero row gets rho = 1.                                    */
+/* ------------------------------------------------------------------------ */
+
+/* pairwise binary64 sum of a[0..n) in index order */
+static double pairwise_sum(const double* a, int64_t n)
+{
+    if (n <= 0) return 0.0;
+    if (n == 1) return a[0];
+    int64_t h = 1;
+    while (h * 2 < n) h *= 2;          /* largest power of two below n */
+    return pairwise_sum(a, h) + pairwise_sum(a + h, n - h);
+}
+
+double orc_pairwise_sum(const double* a, int64_t n) { return pairwise_sum(a, n); }
+
+/* rho of rows [l0, l1) of a row-major [R, ld] input (C columns), blocks of
+ * B elements along the row; also each row's max |x| (rowmax).  Returns 0, or
+ * nonzero for a bad shape or p. */
+int orc_mxnorm_rho(const void* x, int in_dtype, int64_t R, int64_t C, int64_t ld, int B, int p,
+                   double c, int64_t l0, int64_t l1, float* rho, float* rowmax)
+{
+    if (B <= 0 || C % B || (p != 1 && p != 2)) return 1;
+    int64_t K = C / B;
+    double* mp = (double*)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+    for (int64_t l = l0; l < l1; ++l) {
+        float rmax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float m = 0.0f;
+            for (int j = 0; j < B; ++j) {
+                float a = fabsf(load_elem(x, in_dtype, l * ld + k * B + j));
+                if (a > m) m = a;
+            }
+            if (m > rmax) rmax = m;
+            mp[k] = (p == 2) ? (double)m * (double)m : (double)m;
+        }
+        double S = pairwise_sum(mp, K);
+        float r;
+        if (S == 0.0) {
+            r = 1.0f;
+        } else {
+            double mean = S / (double)K;
+            double g = (p == 2) ? sqrt(mean) : mean;
+            double q = c / g;
+            r = (q >= (double)3.4028234663852886e38) ? 3.4028234663852886e38f : (float)q;
+        }
+        rho[l - l0] = r;
+        rowmax[l - l0] = rmax;
+    }
+    (void)R;
+    free(mp);
+    return 0;
+}
