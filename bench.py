@@ -502,7 +502,10 @@ def run_gpu(args, rank, world, device, host):
 
 # ------------------------------------------------------------------------ other workloads
 
-CONFIG_NAMES = ("fprop", "ufp4", "tiny", "wgrad", "dgrad_db")
+CONFIG_NAMES = ("fprop", "ufp4", "mxnorm", "tiny", "wgrad", "dgrad_db")
+# c(2, B) for Gaussian rows, E[max of B |N(0,1)|^2]^(1/2) (B = 32: MXFP4, 16:
+# NVFP4); the kernel's cost does not depend on the value
+MXNORM_C2 = {0: 2.3894571, 1: 2.1329500}
 
 
 def measure_configs(fp4, device, peaks, layer=None, reps=10, only=CONFIG_NAMES):
@@ -551,6 +554,28 @@ def measure_configs(fp4, device, peaks, layer=None, reps=10, only=CONFIG_NAMES):
                 tot_b += e["gbs"] * e["ms"] * 1e6
         out["ufp4_layer_quantize"] = {"calls": uf, "total_ms": tot_ms, "gbs": tot_b / (tot_ms * 1e6),
                                       "frac_hbm": tot_b / (tot_ms * 1e6) / peaks["hbm"]}
+
+    if "mxnorm" in only and layer is not None:
+        # MXNorm fused with the cast ("MXNorm: Reusing MXFP block scales...":
+        # up to 2.4x over RMSNorm + a separate cast on GB200) on the layer's
+        # QKV input, against the cast alone (no rotation) of the same tensor
+        x = layer.linears[0]["t"]["X"]
+        R, C = x.shape
+        ent = {}
+        for fmt, name in ((MX, "mxfp4"), (NV, "nvfp4")):
+            q = fp4.alloc_qtensor(R, C, fmt, device=device)
+            rho = torch.empty(R, dtype=torch.float32, device=device)
+            ws = torch.empty(256, dtype=torch.uint8, device=device)
+            ms = _median_ms(lambda: fp4.mxnorm_quantize(x, fmt, 2, MXNORM_C2[fmt], out=q, rho=rho, workspace=ws),
+                            flush, reps)
+            cast = _median_ms(lambda: fp4.quantize(x, fmt, fp4.FP4_RTNE, fp4.FP4_ROT_NONE, axis=1, out=q, workspace=ws),
+                              flush, reps)
+            reads = 1 if fmt == MX else 2
+            gb = qbytes(x.numel(), 2, fmt, reads=reads) + 4 * R
+            ent[name] = {"ms": ms, "gbs": gb / (ms * 1e6), "frac_hbm": gb / (ms * 1e6) / peaks["hbm"],
+                         "bytes": "%d read%s of x, codes, scales and rho written" % (reads, "s" if reads > 1 else ""),
+                         "cast_alone_ms": cast, "mxnorm_over_cast": ms / cast}
+        out["mxnorm_p2_qkv_input_8192x4096"] = ent
 
     if "tiny" in only:
         d = workloads.tiny_mxfp4()

@@ -271,6 +271,51 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
     return FP4_OK;
 }
 
+fp4_status_t fp4_mxnorm_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                                 fp4_format_t format, fp4_rounding_t rounding, int p, float c, uint64_t seed,
+                                 uint32_t tensor_id, uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                 float* rho, void* workspace, size_t workspace_bytes, void* stream) {
+    fp4_status_t st = check_input(x, in_dtype, rows, cols, ld, FP4_ROT_NONE, 1);
+    if (st != FP4_OK) return st;
+    if (format < FP4_MXFP4 || format > FP4_UFP4) return FP4_ERR_INVALID_ARG;
+    if (rounding != FP4_RTNE && rounding != FP4_SR) return FP4_ERR_INVALID_ARG;
+    if (p != 1 && p != 2) return FP4_ERR_INVALID_ARG;
+    if (!(c > 0.0f) || !(c <= 3.4028234663852886e38f)) return FP4_ERR_INVALID_ARG;   // positive and finite
+    const int64_t blk = (format == FP4_MXFP4) ? 32 : 16;
+    const bool needs_ts = format != FP4_MXFP4;
+    if (rows > 0 && (cols == 0 || cols % blk || cols > 16384)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (needs_ts && !tensor_scale) return FP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!codes || !scales || !rho)) return FP4_ERR_INVALID_ARG;
+    if ((codes && !aligned16(codes)) || (rho && ((uintptr_t)rho & 3u)) ||
+        (tensor_scale && ((uintptr_t)tensor_scale & 3u)))
+        return FP4_ERR_MISALIGNED;
+    if (needs_ts && rows > 0) {
+        if (!workspace || workspace_bytes < 256) return FP4_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    }
+    int dev;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (rows == 0) {
+        if (needs_ts) {
+            static const float one = 1.0f;
+            if (cudaMemcpyAsync(tensor_scale, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return FP4_ERR_CUDA;
+        }
+        return FP4_OK;
+    }
+    unsigned int* amax_word = nullptr;
+    if (needs_ts) {
+        amax_word = static_cast<unsigned int*>(workspace);
+        if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s) != cudaSuccess) return FP4_ERR_CUDA;
+    }
+    if (launch_mxnorm(x, in_dtype == FP4_IN_BF16, rows, cols, ld, format, rounding == FP4_SR, p, (double)c, codes,
+                      scales, needs_ts ? tensor_scale : nullptr, rho, amax_word, make_keys(seed), tensor_id, s) !=
+        cudaSuccess)
+        return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
 fp4_status_t fp4_requantize(const uint8_t* src_codes, const uint8_t* src_scales, const float* src_outer,
                             const float* src_tensor_scale, int64_t lines, int64_t K, fp4_format_t src_format,
                             int src_double_block, fp4_format_t format, fp4_rounding_t rounding,

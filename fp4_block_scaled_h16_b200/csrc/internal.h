@@ -58,6 +58,11 @@ bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int6
 cudaError_t launch_requantize_cols(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db,
                                    cudaStream_t s);
 cudaError_t launch_requant_amax_cols(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s);
+// MXNorm fused with the cast (fp4_mxnorm_quantize); amax_word: a zeroed word
+// (NVFP4 / UFP4 only)
+cudaError_t launch_mxnorm(const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld, int fmt, bool sr, int p,
+                          double c, uint8_t* codes, uint8_t* scales, float* tensor_scale, float* rho,
+                          unsigned int* amax_word, const PhiloxKeys& keys, uint32_t tensor_id, cudaStream_t s);
 // the rotation alone along the rows (fp4_rotate)
 cudaError_t launch_rotate_rows(const void* x, void* y, bool bf16, int64_t rows, int64_t cols, int64_t ld,
                                int64_t ldy, int n, uint32_t sign_mask, cudaStream_t s);

@@ -33,7 +33,7 @@ FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
 
 EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_quantize",
            "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit",
-           "fp4_quantize_noalloc", "fp4_requantize", "fp4_rotate")
+           "fp4_quantize_noalloc", "fp4_requantize", "fp4_rotate", "fp4_mxnorm_quantize")
 
 _P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_uint32, ctypes.c_size_t)
@@ -48,12 +48,14 @@ _lib.fp4_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _I, _U64
 _lib.fp4_quantize_noalloc.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P]
 _lib.fp4_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P, _P,
                                 _P, _SZ, _P]
+_lib.fp4_mxnorm_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, ctypes.c_float, _U64, _U32, _P, _P, _P,
+                                     _P, _P, _SZ, _P]
 _lib.fp4_rotate.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _P, _I64, _P]
 _lib.fp4_gemm.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P]
 _lib.fp4_last_error.argtypes = [_P]
 _lib.fp4_set_wait_limit.argtypes = [_U32]
 _lib.fp4_set_wait_limit.restype = None
-for _f in ("fp4_amax", "fp4_rotate", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
+for _f in ("fp4_amax", "fp4_rotate", "fp4_mxnorm_quantize", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
            "fp4_quantize_workspace_size"):
     getattr(_lib, _f).restype = _I
 
@@ -123,6 +125,31 @@ def rotate(x, rotation, seed=0, out=None, stream=None):
     y = out if out is not None else torch.empty((rows, cols), dtype=x.dtype, device=x.device)
     fp4_rotate(x, in_dtype_of(x), rows, cols, ld, rotation, 1, seed, y, y.stride(0) if rows > 1 else cols, stream)
     return y
+
+
+def fp4_mxnorm_quantize(x, in_dtype, rows, cols, ld, fmt, rounding, p, c, seed, tensor_id, codes, scales,
+                        tensor_scale, rho, workspace, workspace_bytes, stream=None) -> None:
+    _check(_lib.fp4_mxnorm_quantize(_ptr(x), in_dtype, rows, cols, ld, fmt, rounding, p, c, seed, tensor_id,
+                                    _ptr(codes), _ptr(scales), _ptr(tensor_scale), _ptr(rho), _ptr(workspace),
+                                    workspace_bytes, _stream(stream)), "fp4_mxnorm_quantize")
+
+
+def mxnorm_quantize(x, fmt, p, c, rounding=FP4_RTNE, seed=0, tensor_id=0, out=None, rho=None, workspace=None,
+                    stream=None):
+    """MXNorm fused with the cast of a 2-D CUDA tensor along its rows
+    (fp4_mxnorm_quantize): returns the quantized tensor with its "rho" [rows]."""
+    import torch
+    rows, cols = x.shape
+    ld = x.stride(0) if rows > 1 else cols
+    q = out if out is not None else alloc_qtensor(rows, cols, fmt, False, x.device)
+    r = rho if rho is not None else torch.empty(max(rows, 1), dtype=torch.float32, device=x.device)
+    ws_bytes = 0 if fmt == FP4_MXFP4 else 256
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+    fp4_mxnorm_quantize(x, in_dtype_of(x), rows, cols, ld, fmt, rounding, p, c, seed, tensor_id, q["codes"],
+                        q["scales"], q["tensor_scale"], r, workspace if ws_bytes else None, ws_bytes, stream)
+    q["rho"] = r
+    return q
 
 
 def fp4_quantize(x, in_dtype, rows, cols, ld, fmt, rounding, rotation, axis, double_block, seed,

@@ -237,6 +237,45 @@ fp4_status_t fp4_requantize(const uint8_t* src_codes, const uint8_t* src_scales,
                             float* tensor_scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fp4_mxnorm_quantize -- MXNorm fused with the FP4 cast.  "MXNorm: Reusing
+ * MXFP block scales for efficient tensor normalisation", 2. Metodologia: the
+ * inverse RMS of each row t is estimated from the absolute maxima m_tk of the
+ * row's K blocks -- the maxima the cast's block scales come from --
+ *     rho_t = c * ((1/K) sum_k m_tk^p)^(-1/p),   p = 1 or 2,
+ * and the normalised row y = x * rho_t is what gets quantized (the norm's
+ * gain is folded into the next layer's weight, as the page does).
+ *
+ * Arithmetic: m_tk in binary32 over blocks of 32 (MXFP4) or 16 (NVFP4 /
+ * UFP4); the sum of m_tk^p in binary64, pairwise in block order (the sum of a
+ * range is the sum of its two halves, split at the largest power of two
+ * below its length); the mean, the square root (p = 2) and c / g correctly
+ * rounded in binary64, then rounded once to binary32 and saturated at the
+ * largest finite binary32 (an all-zero row: rho = 1); y = RN32(x * rho_t).
+ * y is then quantized along the rows exactly as fp4_quantize would quantize
+ * it with no rotation: MXFP4 block scales, or the NVFP4 / UFP4 block scales
+ * under the tensor scale of y's amax (max_t RN(max|x_t| rho_t)).
+ *
+ *   x, in_dtype, rows, cols, ld  input [rows, ld] row-major, cols valid;
+ *                 cols % 32 (MXFP4) or % 16 (NVFP4, UFP4) == 0, cols <= 16384
+ *   p, c          the mean's order (1 or 2) and the constant c(p, B) > 0
+ *                 (finite): the page takes it from a Monte Carlo simulation;
+ *                 for rows of i.i.d. Gaussian values E[M^p]^(1/p), M the
+ *                 maximum of B independent |N(0, 1)|, makes rho_t tend to
+ *                 1 / RMS (about 2.35 for p = 1 and 2.39 for p = 2, B = 32)
+ *   seed, tensor_id   stochastic rounding, as fp4_quantize (element i = r * cols + c)
+ *   codes, scales, tensor_scale   the quantized y, as fp4_quantize on axis 1
+ *   rho           device float [rows]: rho_t (for the backward pass)
+ *   workspace     NVFP4 / UFP4: >= 256 bytes, 16-byte aligned (the amax of
+ *                 y); MXFP4 needs none
+ * MXFP4 runs one kernel; NVFP4 / UFP4 a statistics kernel (rho, amax of y)
+ * and then the cast.  Errors as fp4_quantize.
+ */
+fp4_status_t fp4_mxnorm_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                                 fp4_format_t format, fp4_rounding_t rounding, int p, float c, uint64_t seed,
+                                 uint32_t tensor_id, uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                 float* rho, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fp4_quantize_noalloc -- fp4_quantize for NVFP4 / UFP4 with the tensor scale
  * taken from an internal amax, for callers that cannot allocate device
  * memory: code running where cudaMalloc is unavailable or forbidden (a plug-in

@@ -157,3 +157,25 @@ def rot(**kw):
 ])
 def test_rotate_host_validation(kw, status):
     assert rot(**kw) == status
+
+
+def mn(**kw):
+    a = dict(x=ADDR, dt=fp4.FP4_IN_BF16, rows=64, cols=256, ld=256, fmt=fp4.FP4_NVFP4, rounding=0, p=2, c=2.0, seed=0,
+             tid=0, codes=ADDR, scales=ADDR, ts=ADDR, rho=ADDR, ws=ADDR, wsb=256)
+    a.update(kw)
+    return fp4._lib.fp4_mxnorm_quantize(a["x"], a["dt"], a["rows"], a["cols"], a["ld"], a["fmt"], a["rounding"],
+                                        a["p"], a["c"], a["seed"], a["tid"], a["codes"], a["scales"], a["ts"],
+                                        a["rho"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dt=4), 1), (dict(fmt=5), 1), (dict(rounding=3), 1), (dict(p=0), 1), (dict(p=3), 1), (dict(c=0.0), 1),
+    (dict(c=-1.0), 1), (dict(c=float("nan")), 1), (dict(c=float("inf")), 1), (dict(ts=None), 1), (dict(rho=None), 1),
+    (dict(codes=None), 1), (dict(ld=128), 1),
+    (dict(cols=248, ld=256), 2), (dict(fmt=fp4.FP4_MXFP4, cols=240, ld=256), 2), (dict(cols=16400, ld=16400), 2),
+    (dict(cols=0), 2),
+    (dict(x=ADDR + 4), 3), (dict(codes=ADDR + 8), 3), (dict(rho=ADDR + 2), 3), (dict(ws=ADDR + 4), 3),
+    (dict(ws=None), 4), (dict(wsb=64), 4),
+])
+def test_mxnorm_host_validation(kw, status):
+    assert mn(**kw) == status
