@@ -508,6 +508,15 @@ CONFIG_NAMES = ("fprop", "ufp4", "mxnorm", "tiny", "wgrad", "dgrad_db")
 MXNORM_C2 = {0: 2.3894571, 1: 2.1329500}
 
 
+def layer_gemm_shapes(layer):
+    """(M, N, K) of the layer's 12 GEMMs."""
+    out = []
+    for lin in layer.linears:
+        for _, ra, rb, _ in GEMMS:
+            out.append((lin["qs"][ra]["lines"], lin["qs"][rb]["lines"], lin["qs"][ra]["K"]))
+    return out
+
+
 def measure_configs(fp4, device, peaks, layer=None, reps=10, only=CONFIG_NAMES):
     """Per-kernel timings of the other workloads: quantize GB/s and GEMM TFLOP/s
     with their fractions of the measured HBM and derived FP4 peaks."""
@@ -541,19 +550,40 @@ def measure_configs(fp4, device, peaks, layer=None, reps=10, only=CONFIG_NAMES):
         out["nvfp4_fprop_qkv_8192x6144x4096"] = fprop_component(fp4, device, flush, peaks, reps)
 
     if "ufp4" in only and layer is not None:
-        # the UFP4 quantizer (levels k * s, k in [-7, 7]) on the layer's operands
-        uf = {}
-        tot_ms = tot_b = 0.0
+        # the UFP4 recipe (levels k * s, k in [-7, 7]) on the layer's operands:
+        # the 24 quantize calls, then the 12 GEMMs.  A UFP4 GEMM runs as an
+        # NVFP4 GEMM over the operands' E2M1 parts, 4x the tensor-core work:
+        # its ceiling is a quarter of the FP4 peak
+        uf, ug = {}, {}
+        tot_ms = tot_b = g_ms = g_flop = 0.0
+        ws = torch.empty(max(fp4.fp4_gemm_workspace_size(UF, False, *g) for g in layer_gemm_shapes(layer)),
+                         dtype=torch.uint8, device=device)
         for lin in layer.linears:
+            qs = []
             for role, c in enumerate(lin["calls"]):
                 x = lin["t"][c["x"]]
-                _, e = quant_entry(x, fmt=UF, rounding=c["rounding"], rotation=fp4.FP4_ROT_H16, axis=c["axis"],
+                q, e = quant_entry(x, fmt=UF, rounding=c["rounding"], rotation=fp4.FP4_ROT_H16, axis=c["axis"],
                                    seed=0, tensor_id=c["tensor_id"])
+                qs.append(q)
                 uf.setdefault(lin["name"], {})[c["name"]] = e
                 tot_ms += e["ms"]
                 tot_b += e["gbs"] * e["ms"] * 1e6
-        out["ufp4_layer_quantize"] = {"calls": uf, "total_ms": tot_ms, "gbs": tot_b / (tot_ms * 1e6),
-                                      "frac_hbm": tot_b / (tot_ms * 1e6) / peaks["hbm"]}
+            for gname, ra, rb, bf16 in GEMMS:
+                M, N, K = qs[ra]["lines"], qs[rb]["lines"], qs[ra]["K"]
+                C = lin["outs"][[g[0] for g in GEMMS].index(gname)]
+                od = BF if bf16 else F32
+                ms = _median_ms(lambda: fp4.gemm(qs[ra], qs[rb], od, out=C, workspace=ws), flush, reps)
+                tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+                ug.setdefault(lin["name"], {})[gname] = {"ms": ms, "tflops": tf, "frac_fp4_over_4": tf / (fp4_peak / 4),
+                                                         "shape": [M, N, K]}
+                g_ms += ms
+                g_flop += 2.0 * M * N * K
+            del qs
+        out["ufp4_layer"] = {"quantize": uf, "quantize_total_ms": tot_ms, "quantize_gbs": tot_b / (tot_ms * 1e6),
+                             "quantize_frac_hbm": tot_b / (tot_ms * 1e6) / peaks["hbm"],
+                             "gemm": ug, "gemm_total_ms": g_ms, "gemm_tflops": g_flop / (g_ms * 1e-3) / 1e12,
+                             "gemm_frac_fp4_over_4": g_flop / (g_ms * 1e-3) / 1e12 / (fp4_peak / 4)}
+        del ws
 
     if "mxnorm" in only and layer is not None:
         # MXNorm fused with the cast ("MXNorm: Reusing MXFP block scales...":

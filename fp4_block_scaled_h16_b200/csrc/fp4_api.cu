@@ -398,16 +398,23 @@ fp4_status_t fp4_requantize(const uint8_t* src_codes, const uint8_t* src_scales,
     return FP4_OK;
 }
 
+fp4_status_t fp4_gemm_workspace_size(fp4_format_t format, int double_block, int64_t M, int64_t N, int64_t K,
+                                     size_t* bytes) {
+    if (!bytes || format < FP4_MXFP4 || format > FP4_UFP4 || M < 0 || N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (double_block != 0 && double_block != 1) return FP4_ERR_INVALID_ARG;
+    *bytes = (format == FP4_UFP4 && !double_block && M > 0 && N > 0 && K > 0)
+                 ? ufp4_split_bytes(M, K) + ufp4_split_bytes(N, K) : 0;
+    return FP4_OK;
+}
+
 fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
                       const uint8_t* a_codes, const uint8_t* a_scales, const float* a_outer,
                       const float* a_tensor_scale,
                       const uint8_t* b_codes, const uint8_t* b_scales, const float* b_outer,
                       const float* b_tensor_scale,
                       int64_t M, int64_t N, int64_t K, void* c, fp4_out_dtype_t out_dtype, int64_t ldc,
-                      void* stream) {
-    if (format != FP4_MXFP4 && format != FP4_NVFP4) {
-        return format == FP4_UFP4 ? FP4_ERR_UNSUPPORTED : FP4_ERR_INVALID_ARG;
-    }
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    if (format < FP4_MXFP4 || format > FP4_UFP4) return FP4_ERR_INVALID_ARG;
     if (double_block != 0 && double_block != 1) return FP4_ERR_INVALID_ARG;
     if (double_block && format != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
@@ -416,15 +423,45 @@ fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
     if (M % 128 || N % 128 || K % 128 || K == 0) return FP4_ERR_UNSUPPORTED_SHAPE;
     if (double_block && K > 8192) return FP4_ERR_UNSUPPORTED_SHAPE;
     if (!a_codes || !a_scales || !b_codes || !b_scales || !c) return FP4_ERR_INVALID_ARG;
-    if (format == FP4_NVFP4 && !double_block && (!a_tensor_scale || !b_tensor_scale)) return FP4_ERR_INVALID_ARG;
+    if (format != FP4_MXFP4 && !double_block && (!a_tensor_scale || !b_tensor_scale)) return FP4_ERR_INVALID_ARG;
     if (double_block && (!a_outer || !b_outer)) return FP4_ERR_INVALID_ARG;
     const int64_t es = out_dtype == FP4_OUT_BF16 ? 2 : 4;
     if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
         !aligned16(c) || (ldc * es) % 16 || (double_block && (!aligned16(a_outer) || !aligned16(b_outer))))
         return FP4_ERR_MISALIGNED;
+    const size_t split_a = format == FP4_UFP4 ? ufp4_split_bytes(M, K) : 0;
+    if (format == FP4_UFP4) {
+        if (!workspace || workspace_bytes < split_a + ufp4_split_bytes(N, K)) return FP4_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    }
     int dev;
     fp4_status_t st;
     if ((st = device_ready(&dev)) != FP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (format == FP4_UFP4) {
+        // A B^T = A1 B1^T + A1 B2^T + A2 B1^T + A2 B2^T with A = A1 + A2, B = B1 + B2
+        // in E2M1 under the same block scales: one NVFP4 GEMM over 4 Kp
+        uint8_t* wa = static_cast<uint8_t*>(workspace);
+        uint8_t* wb = wa + split_a;
+        if (launch_ufp4_split(a_codes, a_scales, M, K, wa, false, s) != cudaSuccess ||
+            launch_ufp4_split(b_codes, b_scales, N, K, wb, true, s) != cudaSuccess)
+            return FP4_ERR_CUDA;
+        const int64_t Kp = (K + 255) / 256 * 256;
+        GemmArgs g{};
+        g.a_codes = wa;
+        g.a_scales = wa + ((size_t)M * (size_t)(2 * Kp) + 1023) / 1024 * 1024;
+        g.a_ts = a_tensor_scale;
+        g.b_codes = wb;
+        g.b_scales = wb + ((size_t)N * (size_t)(2 * Kp) + 1023) / 1024 * 1024;
+        g.b_ts = b_tensor_scale;
+        g.M = M; g.N = N; g.K = 4 * Kp; g.c = c; g.ldc = ldc;
+        g.out_bf16 = out_dtype == FP4_OUT_BF16;
+        g.fmt = FP4_NVFP4;
+        g.db = 0;
+        g.wait_limit = g_wait_limit;
+        if (launch_gemm(g, s) != cudaSuccess) return FP4_ERR_CUDA;
+        return FP4_OK;
+    }
     GemmArgs g{};
     g.a_codes = a_codes; g.a_scales = a_scales; g.a_outer = a_outer; g.a_ts = a_tensor_scale;
     g.b_codes = b_codes; g.b_scales = b_scales; g.b_outer = b_outer; g.b_ts = b_tensor_scale;
@@ -433,7 +470,7 @@ fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
     g.fmt = format;
     g.db = double_block;
     g.wait_limit = g_wait_limit;
-    if (launch_gemm(g, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP4_ERR_CUDA;
+    if (launch_gemm(g, s) != cudaSuccess) return FP4_ERR_CUDA;
     return FP4_OK;
 }
 

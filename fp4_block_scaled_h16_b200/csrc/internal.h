@@ -86,6 +86,12 @@ struct GemmArgs {
     uint32_t wait_limit;
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+// UFP4 operands as two E2M1 parts (ufp4_split.cu): bytes of one operand's
+// split form, and the kernel writing it (codes, then scales at a 1024-byte
+// boundary); b_operand selects the segment order [1 1 2 2] instead of [1 2 1 2]
+size_t ufp4_split_bytes(int64_t L, int64_t K);
+cudaError_t launch_ufp4_split(const uint8_t* codes, const uint8_t* scales, int64_t L, int64_t K, uint8_t* out,
+                              bool b_operand, cudaStream_t s);
 cudaError_t launch_gemm_db(const GemmArgs& g, cudaStream_t s);
 // 2-D TMA map over packed codes [rows, K/2] bytes: box 128 bytes x box_rows, 128-byte swizzle
 bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K, int box_rows);

@@ -33,7 +33,8 @@ FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
 
 EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_quantize",
            "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit",
-           "fp4_quantize_noalloc", "fp4_requantize", "fp4_rotate", "fp4_mxnorm_quantize")
+           "fp4_quantize_noalloc", "fp4_requantize", "fp4_rotate", "fp4_mxnorm_quantize",
+           "fp4_gemm_workspace_size")
 
 _P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_uint32, ctypes.c_size_t)
@@ -51,11 +52,12 @@ _lib.fp4_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _I, 
 _lib.fp4_mxnorm_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, ctypes.c_float, _U64, _U32, _P, _P, _P,
                                      _P, _P, _SZ, _P]
 _lib.fp4_rotate.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _P, _I64, _P]
-_lib.fp4_gemm.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P]
+_lib.fp4_gemm.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P, _SZ, _P]
+_lib.fp4_gemm_workspace_size.argtypes = [_I, _I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]
 _lib.fp4_last_error.argtypes = [_P]
 _lib.fp4_set_wait_limit.argtypes = [_U32]
 _lib.fp4_set_wait_limit.restype = None
-for _f in ("fp4_amax", "fp4_rotate", "fp4_mxnorm_quantize", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
+for _f in ("fp4_amax", "fp4_rotate", "fp4_mxnorm_quantize", "fp4_gemm_workspace_size", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
            "fp4_quantize_workspace_size"):
     getattr(_lib, _f).restype = _I
 
@@ -198,11 +200,19 @@ def fp4_quantize_noalloc(x, in_dtype, rows, cols, ld, fmt, rounding, rotation, a
            "fp4_quantize_noalloc")
 
 
+def fp4_gemm_workspace_size(fmt: int, double_block: bool, M: int, N: int, K: int) -> int:
+    n = _SZ(0)
+    _check(_lib.fp4_gemm_workspace_size(fmt, int(double_block), M, N, K, ctypes.byref(n)), "fp4_gemm_workspace_size")
+    return n.value
+
+
 def fp4_gemm(fmt, double_block, a_codes, a_scales, a_outer, a_tensor_scale, b_codes, b_scales,
-             b_outer, b_tensor_scale, M, N, K, c, out_dtype, ldc, stream=None) -> None:
+             b_outer, b_tensor_scale, M, N, K, c, out_dtype, ldc, workspace=None, workspace_bytes=0,
+             stream=None) -> None:
     _check(_lib.fp4_gemm(fmt, int(double_block), _ptr(a_codes), _ptr(a_scales), _ptr(a_outer),
                          _ptr(a_tensor_scale), _ptr(b_codes), _ptr(b_scales), _ptr(b_outer),
-                         _ptr(b_tensor_scale), M, N, K, _ptr(c), out_dtype, ldc, _stream(stream)),
+                         _ptr(b_tensor_scale), M, N, K, _ptr(c), out_dtype, ldc, _ptr(workspace),
+                         workspace_bytes, _stream(stream)),
            "fp4_gemm")
 
 
@@ -251,8 +261,9 @@ def quantize(x, fmt, rounding=FP4_RTNE, rotation=FP4_ROT_NONE, axis=1, double_bl
     return q
 
 
-def gemm(qa, qb, out_dtype=FP4_OUT_F32, out=None, stream=None):
-    """C = A B^T on two quantized tensors of the same format (lines along K)."""
+def gemm(qa, qb, out_dtype=FP4_OUT_F32, out=None, workspace=None, stream=None):
+    """C = A B^T on two quantized tensors of the same format (lines along K);
+    UFP4 takes a workspace (allocated here when none is given)."""
     import torch
     M, N, K = qa["lines"], qb["lines"], qa["K"]
     if qb["K"] != K or qa["format"] != qb["format"] or qa["double_block"] != qb["double_block"]:
@@ -260,7 +271,10 @@ def gemm(qa, qb, out_dtype=FP4_OUT_F32, out=None, stream=None):
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16 if out_dtype == FP4_OUT_BF16 else torch.float32,
                           device=qa["codes"].device)
+    ws_bytes = fp4_gemm_workspace_size(qa["format"], qa["double_block"], M, N, K)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=qa["codes"].device)
     fp4_gemm(qa["format"], qa["double_block"], qa["codes"], qa["scales"], qa["outer"], qa["tensor_scale"],
              qb["codes"], qb["scales"], qb["outer"], qb["tensor_scale"], M, N, K, out, out_dtype,
-             out.stride(0), stream)
+             out.stride(0), workspace if ws_bytes else None, ws_bytes, stream)
     return out

@@ -308,12 +308,30 @@ fp4_status_t fp4_quantize_noalloc(const void* x, fp4_in_dtype_t in_dtype, int64_
                                   uint8_t* codes, uint8_t* scales, float* tensor_scale, void* stream);
 
 /*
+ * fp4_gemm_workspace_size -- device workspace fp4_gemm needs: for UFP4 the
+ * two operands rewritten as E2M1 parts (see fp4_gemm), about 2 (M + N) K
+ * bytes of codes plus their scales; 0 for MXFP4 and NVFP4.  Returns
+ * FP4_ERR_INVALID_ARG for a bad format or size or a null `bytes`.
+ */
+fp4_status_t fp4_gemm_workspace_size(fp4_format_t format, int double_block, int64_t M, int64_t N, int64_t K,
+                                     size_t* bytes);
+
+/*
  * fp4_gemm -- block-scaled FP4 GEMM on tcgen05 tensor cores:
  *     C[i, j] = alpha_ij * sum_k qA[i, k] qB[j, k] sA[i, k/blk] sB[j, k/blk]
  * with A [M, K] and B [N, K] quantized tensors in the K-major view (lines
  * along K) of the same format, as fp4_quantize writes them:
  *   MXFP4:  alpha = 1, blk = 32 (E8M0 scales);
  *   NVFP4:  alpha = a_tensor_scale * b_tensor_scale, blk = 16 (E4M3);
+ *   UFP4:   as NVFP4, with q the uniform levels k in [-7, 7] ("Ripensare il
+ *           Bias di Shrinkage nel Pretraining di LLM in FP4", Metodologia 2).
+ *           The tensor cores take E2M1 codes only, and 5 and 7 are not E2M1
+ *           values; but every level is a1 + a2 with a1 in {0,1,2,3,4,4,6,6}
+ *           and a2 in {0,0,0,0,0,1,0,1} (both E2M1 under the same block
+ *           scale), so A B^T = A1 B1^T + A1 B2^T + A2 B1^T + A2 B2^T exactly.
+ *           The call writes [A1 A2 A1 A2] and [B1 B1 B2 B2] into the workspace
+ *           (one pass over each operand) and runs one NVFP4 GEMM over 4 K:
+ *           four times the tensor-core work of an NVFP4 GEMM;
  *   double block: alpha varies per 128-element K chunk:
  *           a_outer[i, k/128] * b_outer[j, k/128].
  * This is the Fprop (Y = X W^T), Dgrad (dX = dY W: B = W quantized on
@@ -323,6 +341,8 @@ fp4_status_t fp4_quantize_noalloc(const void* x, fp4_in_dtype_t in_dtype, int64_
  * the GEMM applies no inverse rotation.
  *
  *   c         device, [M, ldc] row-major, fp32 or bf16, ldc >= N
+ *   workspace device, >= fp4_gemm_workspace_size() bytes, 16-byte aligned
+ *             (UFP4 only; NULL and 0 otherwise); contents are scratch
  * Shape rules: M % 128 == 0, N % 128 == 0, K % 128 == 0 (double block: also
  * K <= 8192); ldc * size % 16 == 0.
  * The accumulation is FP32 on the tensor cores.
@@ -333,7 +353,8 @@ fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
                       const uint8_t* b_codes, const uint8_t* b_scales,
                       const float* b_outer, const float* b_tensor_scale,
                       int64_t M, int64_t N, int64_t K,
-                      void* c, fp4_out_dtype_t out_dtype, int64_t ldc, void* stream);
+                      void* c, fp4_out_dtype_t out_dtype, int64_t ldc,
+                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * fp4_last_error -- synchronizes `stream` and returns (and clears) the device

@@ -81,15 +81,20 @@ def test_quantize_host_validation(kw, status):
 
 def g(**kw):
     args = dict(fmt=fp4.FP4_NVFP4, db=0, a=ADDR, sa=ADDR, oa=None, ta=ADDR, b=ADDR, sb=ADDR, ob=None, tb=ADDR,
-                M=256, N=256, K=512, c=ADDR, out=fp4.FP4_OUT_BF16, ldc=256)
+                M=256, N=256, K=512, c=ADDR, out=fp4.FP4_OUT_BF16, ldc=256, ws=None, wsb=0)
     args.update(kw)
     return fp4._lib.fp4_gemm(args["fmt"], args["db"], args["a"], args["sa"], args["oa"], args["ta"], args["b"],
                              args["sb"], args["ob"], args["tb"], args["M"], args["N"], args["K"], args["c"],
-                             args["out"], args["ldc"], None)
+                             args["out"], args["ldc"], args["ws"], args["wsb"], None)
+
+
+UFP4_WS = 2 * (256 * 2 * 512 + 256 * 4 * 512 // 16)     # both operands' split codes + scales at M = N = 256, K = 512
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(fmt=7), 1), (dict(fmt=fp4.FP4_UFP4), 8), (dict(out=3), 1), (dict(ldc=100), 1),
+    (dict(fmt=7), 1), (dict(fmt=fp4.FP4_UFP4), 4), (dict(fmt=fp4.FP4_UFP4, ws=ADDR, wsb=1024), 4),
+    (dict(fmt=fp4.FP4_UFP4, ws=ADDR + 8, wsb=UFP4_WS), 3), (dict(fmt=fp4.FP4_UFP4, ta=None, ws=ADDR, wsb=UFP4_WS), 1),
+    (dict(fmt=fp4.FP4_UFP4, db=1, oa=ADDR, ob=ADDR), 1), (dict(out=3), 1), (dict(ldc=100), 1),
     (dict(M=-128), 1), (dict(a=None), 1), (dict(ta=None), 1), (dict(db=1, fmt=fp4.FP4_MXFP4), 1),
     (dict(M=200), 2), (dict(N=192), 2), (dict(K=320), 2), (dict(K=0), 2),
     (dict(a=ADDR + 8), 3), (dict(ldc=260), 3),
@@ -179,3 +184,13 @@ def mn(**kw):
 ])
 def test_mxnorm_host_validation(kw, status):
     assert mn(**kw) == status
+
+
+def test_gemm_workspace_size():
+    assert fp4.fp4_gemm_workspace_size(fp4.FP4_NVFP4, False, 256, 256, 512) == 0
+    assert fp4.fp4_gemm_workspace_size(fp4.FP4_MXFP4, False, 256, 256, 512) == 0
+    assert fp4.fp4_gemm_workspace_size(fp4.FP4_UFP4, False, 256, 256, 512) == UFP4_WS
+    # K is rounded up to 256 per split part
+    assert fp4.fp4_gemm_workspace_size(fp4.FP4_UFP4, False, 128, 128, 384) == 2 * (128 * 2 * 512 + 128 * 4 * 512 // 16)
+    with pytest.raises(fp4.Fp4Error):
+        fp4.fp4_gemm_workspace_size(9, False, 1, 1, 1)

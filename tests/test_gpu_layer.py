@@ -9,9 +9,9 @@ Per linear, at full size:
     operands, quantized by the CUDA path in NVFP4 and in UFP4 and compared
     bit for bit with the oracle on sampled lines (the oracle takes the tensor
     amax over the whole rotated tensor);
-  * the three NVFP4 GEMMs, including the gate+up Dgrad at K = 28672, the down
-    Fprop at K = 14336 and the Wgrads at K = 8192, compared with the oracle's
-    float64 GEMM on sampled rows and columns within
+  * the three GEMMs in NVFP4 and in UFP4, including the gate+up Dgrad at
+    K = 28672, the down Fprop at K = 14336 and the Wgrads at K = 8192,
+    compared with the oracle's float64 GEMM on sampled rows and columns within
     |C - C64| <= 1e-5 * sum_k |a_ik b_jk| (+ half a bf16 ulp for bf16 out).
 """
 import numpy as np
@@ -59,7 +59,7 @@ def test_layer_linear_full_size(fp4, index):
     host = {k: oracle_input(v) for k, v in d.items()}
     dev = {k: v.cuda() for k, v in d.items()}
     amax = {}
-    nv = {}
+    qs = {}
     for role, (t, axis, sr) in enumerate(workloads.LAYER_OPERANDS):
         if (t, axis) not in amax:
             amax[(t, axis)] = rotated_amax(host[t], axis)
@@ -77,12 +77,9 @@ def test_layer_linear_full_size(fp4, index):
             # g holds the sampled lines only, in the order of `lines`
             assert_quant_equal(g, o, lines=np.arange(len(lines)),
                                what="%s %s axis %d fmt %d" % (name, t, axis, fmt))
-            if fmt == NV:
-                nv[role] = (q, kw)
-            else:
-                del q
-    for gname, ra, rb, out_bf16 in workloads.LAYER_GEMMS:
-        (qa, ka), (qb, kb) = nv[ra], nv[rb]
+            qs[(fmt, role)] = (q, kw)
+    for (fmt, gname, ra, rb, out_bf16) in [(f,) + g for f in (NV, UF) for g in workloads.LAYER_GEMMS]:
+        (qa, ka), (qb, kb) = qs[(fmt, ra)], qs[(fmt, rb)]
         C = fp4.gemm(qa, qb, fp4.FP4_OUT_BF16 if out_bf16 else fp4.FP4_OUT_F32)
         torch.cuda.synchronize()
         assert fp4.fp4_last_error() == fp4.FP4_OK
@@ -94,7 +91,7 @@ def test_layer_linear_full_size(fp4, index):
         C64, bound = oracle.gemm(oa, ob)
         sub = C.float()[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].cpu().numpy()
         assert_within_gemm_bound(sub, C64, bound, out_bf16,
-                                 what="%s %s %s" % (name, gname, (qa["lines"], qb["lines"], qa["K"])))
+                                 what="%s %s fmt %d %s" % (name, gname, fmt, (qa["lines"], qb["lines"], qa["K"])))
         del C
-    del dev, nv
+    del dev, qs
     torch.cuda.empty_cache()

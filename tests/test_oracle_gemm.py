@@ -4,7 +4,9 @@ rational arithmetic on tiny operands that enumerate every 4-bit code.
 The GEMM is C[i, j] = sum_k deq(A)[i, k] * deq(B)[j, k] for A [M, K] and
 B [N, K] quantized along K ("Pre-addestramento ... con MXFP4", Metodologia:
 FP4 operands in the Fprop / Dgrad / Wgrad GEMMs; block scales per 32 (MX) or
-16 (NV) elements, "TetraJet-v2" 2.A for the 16-groups and 128/16 double block).
+16 (NV, UFP4) elements, "TetraJet-v2" 2.A for the 16-groups and 128/16 double
+block; the uniform UFP4 levels of "Ripensare il Bias di Shrinkage nel
+Pretraining di LLM in FP4", Metodologia 2).
 Codes are packed here by hand, element 2j in the low nibble of byte j.
 """
 from fractions import Fraction
@@ -20,6 +22,13 @@ def e2m1_exact(code):
     s, e, m = (code >> 3) & 1, (code >> 1) & 3, code & 1
     mag = Fraction(m, 2) if e == 0 else (1 + Fraction(m, 2)) * Fraction(2) ** (e - 1)
     return -mag if s else mag
+
+
+def ufp4_exact(code):
+    """UFP4 level k * sign, k = code & 7 ("Ripensare il Bias di Shrinkage...",
+    Metodologia 2: levels k s, k in [-7, 7])."""
+    k = Fraction(code & 7)
+    return -k if code & 8 else k
 
 
 def e4m3_exact(code):
@@ -40,7 +49,7 @@ def all_code_rows(rows, K, rng):
 
 
 @pytest.mark.parametrize("fmt,db", [(oracle.MXFP4, False), (oracle.NVFP4, False),
-                                    (oracle.NVFP4, True)])
+                                    (oracle.NVFP4, True), (oracle.UFP4, False)])
 @pytest.mark.parametrize("shape", [(1, 1, 32), (2, 2, 64), (3, 2, 256)])
 def test_gemm_oracle_brute_force(fmt, db, shape):
     M, N, K = shape
@@ -69,7 +78,8 @@ def test_gemm_oracle_brute_force(fmt, db, shape):
     C64, bound = oracle.gemm(qt(ca, sa, ta, oa), qt(cb, sb, tb, ob))
 
     def ref(codes, scales, ts, outer, i, k):
-        v = e2m1_exact(int(codes[i, k])) * dec(scales[i, k // blk])
+        elem = ufp4_exact if fmt == oracle.UFP4 else e2m1_exact
+        v = elem(int(codes[i, k])) * dec(scales[i, k // blk])
         if fmt != oracle.MXFP4:
             v *= Fraction(float(outer[i, k // 128])) if db else Fraction(float(ts))
         return v
