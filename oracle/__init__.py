@@ -90,6 +90,7 @@ def lib():
         L.orc_pairwise_sum.argtypes = [P, i64]
         L.orc_pairwise_sum.restype = ctypes.c_double
         L.orc_mxnorm_rho.argtypes = [P, i32, i64, i64, i64, i32, i32, ctypes.c_double, i64, i64, P, P]
+        L.orc_fp8_encode_array.argtypes = [P, i64, f32, P]
         _lib = L
     return _lib
 
@@ -379,3 +380,71 @@ def mxnorm_constant(p: int, block: int) -> float:
     f = lambda m: p * m ** (p - 1) * (1.0 - special.erf(m / np.sqrt(2.0)) ** block)
     val, _ = integrate.quad(f, 0.0, np.inf, epsabs=1e-13, epsrel=1e-12, limit=200)
     return float(val ** (1.0 / p))
+
+
+# --------------------------------------------------------------------------- OutControl
+
+def outctl_channels(x: np.ndarray, p: float) -> np.ndarray:
+    """The top p of the columns (channels) of a calibration tensor by max |x|,
+    ceil(p * cols) of them, ties to the lower index, in ascending order
+    ("TetraJet-v2" 2.C: the channels with consistently large norms, chosen in
+    a short calibration window and then kept fixed)."""
+    a = np.abs(widen(np.ascontiguousarray(x))).max(axis=0)
+    n = int(np.ceil(p * a.shape[0]))
+    order = np.lexsort((np.arange(a.shape[0]), -a.astype(np.float64)))   # by amax descending, then index
+    return np.sort(order[:n]).astype(np.int32)
+
+
+def fp8_scale(amax: float) -> float:
+    """The FP8 tensor scale amax / 448 in binary32 (1 if that is 0)."""
+    s = np.float32(np.float32(amax) / np.float32(448.0))
+    return float(s) if s > 0 else 1.0
+
+
+def fp8_quantize(x: np.ndarray, K8: int, scale: float | None = None) -> dict:
+    """E4M3 of the [R, n] binary32 tensor x under one tensor scale, the columns
+    zero-padded to K8: codes [R, K8] (sign in bit 7), its scale and amax."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    R, n = x.shape
+    amax = float(np.abs(x).max()) if x.size else 0.0
+    s8 = fp8_scale(amax) if scale is None else scale
+    codes = np.zeros((R, K8), np.uint8)
+    if x.size:
+        tmp = np.zeros((R, n), np.uint8)
+        lib().orc_fp8_encode_array(_ptr(x), x.size, s8, _ptr(tmp))
+        codes[:, :n] = tmp
+    return dict(codes=codes, scale=s8, amax=amax, K=K8)
+
+
+def fp8_dequantize(q: dict) -> np.ndarray:
+    """Exact float64 values q * s8 of an FP8 tensor."""
+    c = q["codes"]
+    mag = np.vectorize(lambda b: lib().orc_e4m3_value(int(b) & 0x7F), otypes=[np.float64])(np.arange(256))
+    sign = np.where(np.arange(256) & 0x80, -1.0, 1.0)
+    table = mag * sign
+    return table[c] * np.float64(q["scale"])
+
+
+def outctl_quantize(x: np.ndarray, channels: np.ndarray, K8: int, fmt: int = NVFP4, rounding: int = RTNE,
+                    rotation: int = ROT_NONE, seed: int = 0, tensor_id: int = 0, lines=None) -> dict:
+    """OutControl's split of one operand along its channels (columns): the FP4
+    part is x with the channels set to zero, quantized as `quantize` does; the
+    FP8 part is x[:, channels] in E4M3 under its own tensor scale."""
+    xf = widen(np.ascontiguousarray(x)).copy()
+    ch = np.asarray(channels, dtype=np.int64)
+    gathered = xf[:, ch].astype(np.float32)
+    xf[:, ch] = 0.0
+    q4 = quantize(xf, fmt, rounding=rounding, rotation=rotation, axis=1, seed=seed, tensor_id=tensor_id,
+                  lines=lines)
+    q8 = fp8_quantize(gathered, K8)
+    if lines is not None:
+        q8["codes"] = q8["codes"][np.asarray(lines)]
+    return dict(fp4=q4, fp8=q8)
+
+
+def gemm_outctl(a: dict, b: dict):
+    """C64 = deq(A4) deq(B4)^T + deq(A8) deq(B8)^T in float64, and the bound
+    sum_k |a b| over both parts."""
+    C4, b4 = gemm(a["fp4"], b["fp4"])
+    a8, b8 = fp8_dequantize(a["fp8"]), fp8_dequantize(b["fp8"])
+    return C4 + a8 @ b8.T, b4 + np.abs(a8) @ np.abs(b8).T

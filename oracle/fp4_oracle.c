@@ -477,3 +477,22 @@ int orc_mxnorm_rho(const void* x, int in_dtype, int64_t R, int64_t C, int64_t ld
     free(mp);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* OutControl's high-precision channels ("TetraJet-v2" 2.C: the top p% of    */
+/* activation channels, fixed after a calibration window, kept in FP8 for     */
+/* the forward and backward passes).  Readings: FP8 is E4M3 under one FP32    */
+/* tensor scale s8 = amax / 448 (1 if that is 0); a value x is coded as       */
+/* E4M3_rne_satfinite(x / s8), the division one IEEE binary32 operation, the  */
+/* sign kept (-0 -> code 0x80).                                               */
+/* ------------------------------------------------------------------------ */
+
+/* E4M3 codes of in[i] / s8 (binary32 division), sign in bit 7 */
+void orc_fp8_encode_array(const float* in, int64_t n, float s8, uint8_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        float v = in[i] / s8;
+        uint8_t mag = orc_e4m3_encode(fabsf(v));
+        out[i] = (uint8_t)((signbit(v) ? 0x80u : 0u) | mag);
+    }
+}
