@@ -502,7 +502,7 @@ def run_gpu(args, rank, world, device, host):
 
 # ------------------------------------------------------------------------ other workloads
 
-CONFIG_NAMES = ("fprop", "ufp4", "mxnorm", "tiny", "wgrad", "dgrad_db")
+CONFIG_NAMES = ("fprop", "ufp4", "mxnorm", "outctl", "tiny", "wgrad", "dgrad_db")
 # c(2, B) for Gaussian rows, E[max of B |N(0,1)|^2]^(1/2) (B = 32: MXFP4, 16:
 # NVFP4); the kernel's cost does not depend on the value
 MXNORM_C2 = {0: 2.3894571, 1: 2.1329500}
@@ -606,6 +606,32 @@ def measure_configs(fp4, device, peaks, layer=None, reps=10, only=CONFIG_NAMES):
                          "bytes": "%d read%s of x, codes, scales and rho written" % (reads, "s" if reads > 1 else ""),
                          "cast_alone_ms": cast, "mxnorm_over_cast": ms / cast}
         out["mxnorm_p2_qkv_input_8192x4096"] = ent
+
+    if "outctl" in only:
+        # OutControl ("TetraJet-v2" 2.C) on the QKV Fprop: calibration on X,
+        # the top 10% channels in FP8 (E4M3), the rest NVFP4; split X and W,
+        # then the split GEMM (two TMEM accumulators)
+        d = workloads.nvfp4_fprop_qkv(seed=0)
+        X, W = d["X"].to(device), d["W"].to(device)
+        M, K = X.shape
+        N = W.shape[0]
+        ch = fp4.outctl_channels(fp4.channel_amax(X), 0.10)
+        qx, qw = fp4.outctl_quantize(X, ch), fp4.outctl_quantize(W, ch)
+        K8 = qx["fp8"]["K"]
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        sq_x = _median_ms(lambda: fp4.outctl_quantize(X, ch, out=qx), flush, reps)
+        sq_w = _median_ms(lambda: fp4.outctl_quantize(W, ch, out=qw), flush, reps)
+        g = _median_ms(lambda: fp4.gemm_outctl(qx, qw, BF, out=C), flush, reps)
+        flop_useful, flop_run = 2.0 * M * N * K, 2.0 * M * N * (K + K8)
+        out["outcontrol_fprop_qkv_8192x6144x4096"] = {
+            "channels_fp8": int(ch.numel()), "K8": int(K8),
+            "split_X_ms": sq_x, "split_W_ms": sq_w,
+            "split_X_gbs": (qbytes(M * K, 2, NV, reads=2) + M * K8 + 2 * M * ch.numel()) / (sq_x * 1e6),
+            "gemm_ms": g, "gemm_tflops_useful": flop_useful / (g * 1e-3) / 1e12,
+            "gemm_tflops_run": flop_run / (g * 1e-3) / 1e12,
+            "gemm_frac_fp4_run": flop_run / (g * 1e-3) / 1e12 / fp4_peak,
+            "note": "FP8 MMAs run at half the FP4 rate; 'run' counts the FP4 and FP8 MACs the kernel issues"}
+        del X, W, qx, qw, C
 
     if "tiny" in only:
         d = workloads.tiny_mxfp4()

@@ -316,6 +316,125 @@ fp4_status_t fp4_mxnorm_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t
     return FP4_OK;
 }
 
+fp4_status_t fp4_channel_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                              float* amax_out, void* stream) {
+    fp4_status_t st = check_input(x, in_dtype, rows, cols, ld, FP4_ROT_NONE, 1);
+    if (st != FP4_OK) return st;
+    if (cols > 0 && !amax_out) return FP4_ERR_INVALID_ARG;
+    if (amax_out && ((uintptr_t)amax_out & 3u)) return FP4_ERR_MISALIGNED;
+    int dev;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cols == 0) return FP4_OK;
+    if (cudaMemsetAsync(amax_out, 0, (size_t)cols * sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
+    if (rows == 0) return FP4_OK;
+    if (launch_channel_amax(x, in_dtype == FP4_IN_BF16, rows, cols, ld, amax_out, s) != cudaSuccess)
+        return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
+// workspace of fp4_outctl_quantize: [0, 256) the FP4 part's amax and grid
+// count, [256, 272) the FP8 part's amax, then the channel mask
+static size_t outctl_ws_bytes(int64_t cols) {
+    return 272 + (size_t)((cols + 127) / 128) * 16;
+}
+
+fp4_status_t fp4_outctl_workspace_size(int64_t cols, size_t* bytes) {
+    if (!bytes || cols < 0) return FP4_ERR_INVALID_ARG;
+    *bytes = outctl_ws_bytes(cols);
+    return FP4_OK;
+}
+
+fp4_status_t fp4_outctl_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                                 const int32_t* channels, int64_t n_channels, int64_t k8, fp4_rounding_t rounding,
+                                 fp4_rotation_t rotation, uint64_t seed, uint32_t tensor_id, uint8_t* codes,
+                                 uint8_t* scales, float* tensor_scale, uint8_t* codes8, float* scale8,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    fp4_status_t st = check_input(x, in_dtype, rows, cols, ld, rotation, 1);
+    if (st != FP4_OK) return st;
+    if (rounding != FP4_RTNE && rounding != FP4_SR) return FP4_ERR_INVALID_ARG;
+    if (n_channels < 0 || k8 < 0 || n_channels > k8 || n_channels > cols) return FP4_ERR_INVALID_ARG;
+    if (n_channels > 0 && !channels) return FP4_ERR_INVALID_ARG;
+    if (cols % 16 || k8 % 128) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!tensor_scale || !scale8) return FP4_ERR_INVALID_ARG;
+    const bool empty = rows == 0 || cols == 0;
+    if (!empty && (!codes || !scales)) return FP4_ERR_INVALID_ARG;
+    if (rows > 0 && k8 > 0 && !codes8) return FP4_ERR_INVALID_ARG;
+    if ((codes && !aligned16(codes)) || (codes8 && !aligned16(codes8)) || ((uintptr_t)tensor_scale & 3u) ||
+        ((uintptr_t)scale8 & 3u) || (channels && ((uintptr_t)channels & 3u)))
+        return FP4_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < outctl_ws_bytes(cols)) return FP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    int dev;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, outctl_ws_bytes(cols), s) != cudaSuccess) return FP4_ERR_CUDA;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    unsigned int* amax8 = reinterpret_cast<unsigned int*>(ws + 256);
+    uint32_t* mask = reinterpret_cast<uint32_t*>(ws + 272);
+    const bool bf16 = in_dtype == FP4_IN_BF16;
+    if (empty) {
+        static const float one = 1.0f;
+        if (cudaMemcpyAsync(tensor_scale, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(scale8, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return FP4_ERR_CUDA;
+        return FP4_OK;
+    }
+    if (launch_channel_mask(channels, n_channels, cols, mask, s) != cudaSuccess) return FP4_ERR_CUDA;
+    // the FP4 part: NVFP4 along the rows with the channels read as +0
+    QuantArgs a{};
+    a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
+    a.L = rows; a.K = cols;
+    a.nb4 = ((cols / 16) + 3) / 4;
+    a.codes = codes; a.scales = scales;
+    a.tensor_scale_out = tensor_scale;
+    a.keys = make_keys(seed);
+    a.tensor_id = tensor_id;
+    a.sign_mask = sign_mask_of(rotation, seed);
+    a.err = device_error_word();
+    a.wait_limit = g_wait_limit;
+    a.amax_out = reinterpret_cast<unsigned int*>(ws);
+    a.grid_count = reinterpret_cast<unsigned int*>(ws) + 1;
+    a.amax_in = reinterpret_cast<const float*>(ws);
+    a.chan_mask = mask;
+    if (launch_quantize_fused(a, bf16, FP4_NVFP4, rounding == FP4_SR, rot_size(rotation), 1, s) != cudaSuccess)
+        return FP4_ERR_CUDA;
+    // the FP8 part
+    if (launch_fp8_gather(x, bf16, rows, cols, ld, channels, n_channels, k8, amax8, codes8, scale8, s) != cudaSuccess)
+        return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
+fp4_status_t fp4_gemm_outctl(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_tensor_scale,
+                             const uint8_t* b_codes, const uint8_t* b_scales, const float* b_tensor_scale,
+                             const uint8_t* a8_codes, const float* a8_scale, const uint8_t* b8_codes,
+                             const float* b8_scale, int64_t M, int64_t N, int64_t K, int64_t K8, void* c,
+                             fp4_out_dtype_t out_dtype, int64_t ldc, void* stream) {
+    if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0 || K8 < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return FP4_OK;
+    if (M % 128 || N % 128 || K % 128 || K == 0 || K8 % 128) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !c || !a_tensor_scale || !b_tensor_scale)
+        return FP4_ERR_INVALID_ARG;
+    if (K8 > 0 && (!a8_codes || !b8_codes || !a8_scale || !b8_scale)) return FP4_ERR_INVALID_ARG;
+    const int64_t es = out_dtype == FP4_OUT_BF16 ? 2 : 4;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
+        !aligned16(c) || (ldc * es) % 16 || (K8 > 0 && (!aligned16(a8_codes) || !aligned16(b8_codes))))
+        return FP4_ERR_MISALIGNED;
+    int dev;
+    fp4_status_t st;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    OutctlGemmArgs g{};
+    g.a_codes = a_codes; g.a_scales = a_scales; g.a_ts = a_tensor_scale;
+    g.b_codes = b_codes; g.b_scales = b_scales; g.b_ts = b_tensor_scale;
+    g.a8_codes = a8_codes; g.a8_scale = a8_scale; g.b8_codes = b8_codes; g.b8_scale = b8_scale;
+    g.M = M; g.N = N; g.K = K; g.K8 = K8; g.c = c; g.ldc = ldc;
+    g.out_bf16 = out_dtype == FP4_OUT_BF16;
+    g.wait_limit = g_wait_limit;
+    if (launch_gemm_outctl(g, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
 fp4_status_t fp4_requantize(const uint8_t* src_codes, const uint8_t* src_scales, const float* src_outer,
                             const float* src_tensor_scale, int64_t lines, int64_t K, fp4_format_t src_format,
                             int src_double_block, fp4_format_t format, fp4_rounding_t rounding,

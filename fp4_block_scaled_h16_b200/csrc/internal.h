@@ -28,6 +28,9 @@ struct QuantArgs {
     uint32_t div_m, div_l;      // multiply-shift division by the units per line
     unsigned int* err;          // device error word (a bounded wait that ran out)
     uint32_t wait_limit;        // polls of a bounded wait (fp4_set_wait_limit)
+    // row axis only: channels (columns) whose bit is set read as +0 (OutControl's
+    // FP8 channels, taken out of the FP4 part); NULL for none
+    const uint32_t* chan_mask;
     // re-quantization (fp4_requantize): the source is a quantized tensor whose
     // lines are the rows of the logical [rows, cols] input; x is unused
     const uint8_t* src_codes;   // [rows, cols/2]
@@ -86,6 +89,31 @@ struct GemmArgs {
     uint32_t wait_limit;
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+// OutControl (outctl.cu, gemm_outctl.cu)
+cudaError_t launch_channel_amax(const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld, float* out,
+                                cudaStream_t s);
+cudaError_t launch_channel_mask(const int32_t* ch, int64_t n, int64_t cols, uint32_t* mask, cudaStream_t s);
+cudaError_t launch_fp8_gather(const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld, const int32_t* ch,
+                              int64_t n, int64_t k8, unsigned int* amax_word, uint8_t* codes, float* scale,
+                              cudaStream_t s);
+struct OutctlGemmArgs {
+    const uint8_t* a_codes;
+    const uint8_t* a_scales;
+    const float* a_ts;
+    const uint8_t* b_codes;
+    const uint8_t* b_scales;
+    const float* b_ts;
+    const uint8_t* a8_codes;
+    const float* a8_scale;
+    const uint8_t* b8_codes;
+    const float* b8_scale;
+    int64_t M, N, K, K8;
+    void* c;
+    int64_t ldc;
+    int out_bf16;
+    uint32_t wait_limit;
+};
+cudaError_t launch_gemm_outctl(const OutctlGemmArgs& g, cudaStream_t s);
 // UFP4 operands as two E2M1 parts (ufp4_split.cu): bytes of one operand's
 // split form, and the kernel writing it (codes, then scales at a 1024-byte
 // boundary); b_operand selects the segment order [1 1 2 2] instead of [1 2 1 2]

@@ -264,6 +264,15 @@ quant_rows_kernel(const QuantArgs a, const RowStages st) {
 #pragma unroll
             for (int e = 0; e < U; ++e) v[e] = 0.0f;
         }
+        if (a.chan_mask && active) {
+            // channels taken out of this tensor (OutControl) read as +0
+            const int64_t c0 = j * U;
+            uint32_t mw = __ldg(a.chan_mask + (c0 >> 5));
+            if (U == 16) mw >>= (uint32_t)(c0 & 16);
+#pragma unroll
+            for (int e = 0; e < U; ++e)
+                if ((mw >> e) & 1u) v[e] = 0.0f;
+        }
         if (AMAX_ONLY || (FUSED && it < n)) {
             tmax = unit_rotated_absmax<U, ROT, SIGNS>(v, a.sign_mask, tmax);
             continue;

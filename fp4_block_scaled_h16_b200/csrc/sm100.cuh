@@ -144,6 +144,23 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uin
                  ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb) : "memory");
 }
 
+// D(tmem) (+)= A(smem) x B(smem)^T with E4M3 operands (kind::f8f6f4, no
+// block scales, K = 32 per instruction), FP32 accumulate; no output lane is
+// disabled (the four-word lane mask is zero)
+__device__ __forceinline__ void mma_f8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+                 ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+                 : "memory");
+}
+
+// instruction descriptor of kind::f8f6f4 with E4M3 x E4M3 -> F32, both
+// operands K-major, M = 128: D format F32 (bits 4-5 = 1), A and B format
+// E4M3 (0), N / 8 at bit 17, M / 16 at bit 24
+__host__ __device__ constexpr uint32_t idesc_f8_e4m3(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
 // instruction descriptor of the block-scaled MMA (M = 128, K = 64, both
 // operands E2M1 and K-major, FP32 accumulate)
 __host__ __device__ constexpr uint32_t idesc_block_scaled(int n, bool ue8m0, uint32_t a_sf_id, uint32_t b_sf_id) {

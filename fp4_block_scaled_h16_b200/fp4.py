@@ -34,7 +34,8 @@ FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
 EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_quantize",
            "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit",
            "fp4_quantize_noalloc", "fp4_requantize", "fp4_rotate", "fp4_mxnorm_quantize",
-           "fp4_gemm_workspace_size")
+           "fp4_gemm_workspace_size", "fp4_channel_amax", "fp4_outctl_workspace_size", "fp4_outctl_quantize",
+           "fp4_gemm_outctl")
 
 _P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_uint32, ctypes.c_size_t)
@@ -51,13 +52,19 @@ _lib.fp4_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _I, 
                                 _P, _SZ, _P]
 _lib.fp4_mxnorm_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, ctypes.c_float, _U64, _U32, _P, _P, _P,
                                      _P, _P, _SZ, _P]
+_lib.fp4_channel_amax.argtypes = [_P, _I, _I64, _I64, _I64, _P, _P]
+_lib.fp4_outctl_workspace_size.argtypes = [_I64, ctypes.POINTER(_SZ)]
+_lib.fp4_outctl_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I64, _I64, _I, _I, _U64, _U32, _P, _P, _P, _P, _P,
+                                     _P, _SZ, _P]
+_lib.fp4_gemm_outctl.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _I, _I64, _P]
 _lib.fp4_rotate.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _P, _I64, _P]
 _lib.fp4_gemm.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P, _SZ, _P]
 _lib.fp4_gemm_workspace_size.argtypes = [_I, _I, _I64, _I64, _I64, ctypes.POINTER(_SZ)]
 _lib.fp4_last_error.argtypes = [_P]
 _lib.fp4_set_wait_limit.argtypes = [_U32]
 _lib.fp4_set_wait_limit.restype = None
-for _f in ("fp4_amax", "fp4_rotate", "fp4_mxnorm_quantize", "fp4_gemm_workspace_size", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
+for _f in ("fp4_amax", "fp4_rotate", "fp4_mxnorm_quantize", "fp4_gemm_workspace_size", "fp4_channel_amax",
+           "fp4_outctl_workspace_size", "fp4_outctl_quantize", "fp4_gemm_outctl", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
            "fp4_quantize_workspace_size"):
     getattr(_lib, _f).restype = _I
 
@@ -277,4 +284,87 @@ def gemm(qa, qb, out_dtype=FP4_OUT_F32, out=None, workspace=None, stream=None):
     fp4_gemm(qa["format"], qa["double_block"], qa["codes"], qa["scales"], qa["outer"], qa["tensor_scale"],
              qb["codes"], qb["scales"], qb["outer"], qb["tensor_scale"], M, N, K, out, out_dtype,
              out.stride(0), workspace if ws_bytes else None, ws_bytes, stream)
+    return out
+
+
+# --------------------------------------------------------------------------- OutControl
+
+def fp4_channel_amax(x, in_dtype, rows, cols, ld, amax_out, stream=None) -> None:
+    _check(_lib.fp4_channel_amax(_ptr(x), in_dtype, rows, cols, ld, _ptr(amax_out), _stream(stream)),
+           "fp4_channel_amax")
+
+
+def fp4_outctl_workspace_size(cols: int) -> int:
+    n = _SZ(0)
+    _check(_lib.fp4_outctl_workspace_size(cols, ctypes.byref(n)), "fp4_outctl_workspace_size")
+    return n.value
+
+
+def fp4_outctl_quantize(x, in_dtype, rows, cols, ld, channels, n_channels, k8, rounding, rotation, seed, tensor_id,
+                        codes, scales, tensor_scale, codes8, scale8, workspace, workspace_bytes, stream=None) -> None:
+    _check(_lib.fp4_outctl_quantize(_ptr(x), in_dtype, rows, cols, ld, _ptr(channels), n_channels, k8, rounding,
+                                    rotation, seed, tensor_id, _ptr(codes), _ptr(scales), _ptr(tensor_scale),
+                                    _ptr(codes8), _ptr(scale8), _ptr(workspace), workspace_bytes, _stream(stream)),
+           "fp4_outctl_quantize")
+
+
+def fp4_gemm_outctl(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, a8_codes, a8_scale, b8_codes, b8_scale,
+                    M, N, K, K8, c, out_dtype, ldc, stream=None) -> None:
+    _check(_lib.fp4_gemm_outctl(_ptr(a_codes), _ptr(a_scales), _ptr(a_ts), _ptr(b_codes), _ptr(b_scales), _ptr(b_ts),
+                                _ptr(a8_codes), _ptr(a8_scale), _ptr(b8_codes), _ptr(b8_scale), M, N, K, K8, _ptr(c),
+                                out_dtype, ldc, _stream(stream)), "fp4_gemm_outctl")
+
+
+def channel_amax(x, stream=None):
+    """max over rows of |x[:, c]| for a 2-D CUDA tensor (fp4_channel_amax)."""
+    import torch
+    rows, cols = x.shape
+    out = torch.empty(max(cols, 1), dtype=torch.float32, device=x.device)
+    fp4_channel_amax(x, in_dtype_of(x), rows, cols, x.stride(0) if rows > 1 else cols, out, stream)
+    return out[:cols]
+
+
+def outctl_channels(amax, p: float):
+    """Calibration: the ceil(p * cols) channels with the largest amax (ties to
+    the lower index), in ascending order, as a device int32 tensor."""
+    import math
+    import torch
+    n = math.ceil(p * amax.numel())
+    order = torch.sort(-amax, stable=True).indices[:n]
+    return torch.sort(order).values.to(torch.int32)
+
+
+def outctl_quantize(x, channels, k8=None, rounding=FP4_RTNE, rotation=FP4_ROT_NONE, seed=0, tensor_id=0,
+                    out=None, stream=None):
+    """The OutControl split of a 2-D CUDA tensor along its channels
+    (fp4_outctl_quantize): {"fp4": NVFP4 qtensor, "fp8": {"codes", "scale", "K"}}."""
+    import torch
+    rows, cols = x.shape
+    n = channels.numel()
+    k8 = (n + 127) // 128 * 128 if k8 is None else k8
+    o = out if out is not None else dict(
+        fp4=alloc_qtensor(rows, cols, FP4_NVFP4, False, x.device),
+        fp8=dict(codes=torch.empty((rows, max(k8, 1)), dtype=torch.uint8, device=x.device),
+                 scale=torch.empty(1, dtype=torch.float32, device=x.device), K=k8))
+    ws = torch.empty(fp4_outctl_workspace_size(cols), dtype=torch.uint8, device=x.device)
+    q4, q8 = o["fp4"], o["fp8"]
+    fp4_outctl_quantize(x, in_dtype_of(x), rows, cols, x.stride(0) if rows > 1 else cols, channels, n, k8, rounding,
+                        rotation, seed, tensor_id, q4["codes"], q4["scales"], q4["tensor_scale"], q8["codes"],
+                        q8["scale"], ws, ws.numel(), stream)
+    return o
+
+
+def gemm_outctl(qa, qb, out_dtype=FP4_OUT_F32, out=None, stream=None):
+    """C = A B^T on two OutControl-split operands (fp4_gemm_outctl)."""
+    import torch
+    a4, b4, a8, b8 = qa["fp4"], qb["fp4"], qa["fp8"], qb["fp8"]
+    M, N, K, K8 = a4["lines"], b4["lines"], a4["K"], a8["K"]
+    if b4["K"] != K or b8["K"] != K8:
+        raise ValueError("operands must share K and the FP8 width")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16 if out_dtype == FP4_OUT_BF16 else torch.float32,
+                          device=a4["codes"].device)
+    fp4_gemm_outctl(a4["codes"], a4["scales"], a4["tensor_scale"], b4["codes"], b4["scales"], b4["tensor_scale"],
+                    a8["codes"], a8["scale"], b8["codes"], b8["scale"], M, N, K, K8, out, out_dtype, out.stride(0),
+                    stream)
     return out

@@ -276,6 +276,70 @@ fp4_status_t fp4_mxnorm_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t
                                  float* rho, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * OutControl ("TetraJet-v2", 2.C): a few activation channels carry outliers
+ * and do so consistently, so the top p% of the channels (the columns of the
+ * activation, i.e. the GEMM's contraction index), chosen once in a short
+ * calibration window, are kept in FP8 for the forward and backward passes and
+ * the rest stays FP4.  The split of a [rows, cols] operand:
+ *   FP4 part   the operand with those channels set to +0, quantized to NVFP4
+ *              along the rows exactly as fp4_quantize does (so the outliers
+ *              no longer set its tensor and block scales);
+ *   FP8 part   the operand's channels, gathered in list order into
+ *              [rows, k8] E4M3 codes (sign in bit 7, zero past the list) under
+ *              one FP32 tensor scale s8 = amax / 448 (1 if that is 0):
+ *              code = E4M3_rne_satfinite(RN(x / s8)).
+ * Both GEMM operands are split with the same channel list, and
+ *     C = a4 b4 (FP4 product) + s8A s8B (FP8 product)
+ * runs in one kernel (fp4_gemm_outctl).
+ */
+
+/*
+ * fp4_channel_amax -- the calibration statistic: amax_out[c] = max_r |x[r, c]|
+ * for a [rows, ld] row-major input (device float [cols], overwritten).  The
+ * caller picks its top channels from it.
+ */
+fp4_status_t fp4_channel_amax(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                              float* amax_out, void* stream);
+
+/* fp4_outctl_workspace_size -- workspace bytes of fp4_outctl_quantize for `cols` columns. */
+fp4_status_t fp4_outctl_workspace_size(int64_t cols, size_t* bytes);
+
+/*
+ * fp4_outctl_quantize -- the OutControl split of one operand (above).
+ *   x, in_dtype, rows, cols, ld   input [rows, ld] row-major; cols % 16 == 0
+ *   channels, n_channels  device int32 [n_channels], ascending, unique, in
+ *                 [0, cols) (an index outside is skipped and reported by
+ *                 fp4_last_error as FP4_ERR_INVALID_ARG)
+ *   k8            columns of the FP8 part: n_channels <= k8, k8 % 128 == 0
+ *   rounding, rotation, seed, tensor_id   of the FP4 part, as fp4_quantize
+ *   codes, scales, tensor_scale   the FP4 part, as fp4_quantize on axis 1
+ *   codes8        device uint8 [rows, k8], 16-byte aligned
+ *   scale8        device float, receives s8
+ *   workspace     >= fp4_outctl_workspace_size(cols) bytes, 16-byte aligned
+ */
+fp4_status_t fp4_outctl_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                                 const int32_t* channels, int64_t n_channels, int64_t k8, fp4_rounding_t rounding,
+                                 fp4_rotation_t rotation, uint64_t seed, uint32_t tensor_id, uint8_t* codes,
+                                 uint8_t* scales, float* tensor_scale, uint8_t* codes8, float* scale8,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fp4_gemm_outctl -- C = a4 b4 sum_k qA qB sA sB + s8A s8B sum_k8 eA eB for the
+ * split operands A [M, K] / [M, K8] and B [N, K] / [N, K8] of
+ * fp4_outctl_quantize: the NVFP4 product and the E4M3 product (tcgen05
+ * kind::f8f6f4) accumulate in two TMEM accumulators of one tile, and each
+ * output element is formed and rounded once.
+ *   c, out_dtype, ldc   as fp4_gemm
+ * Shape rules: M, N, K multiples of 128 (K > 0), K8 a multiple of 128 (0: no
+ * FP8 part, the FP8 pointers may be NULL); code pointers 16-byte aligned.
+ */
+fp4_status_t fp4_gemm_outctl(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_tensor_scale,
+                             const uint8_t* b_codes, const uint8_t* b_scales, const float* b_tensor_scale,
+                             const uint8_t* a8_codes, const float* a8_scale, const uint8_t* b8_codes,
+                             const float* b8_scale, int64_t M, int64_t N, int64_t K, int64_t K8, void* c,
+                             fp4_out_dtype_t out_dtype, int64_t ldc, void* stream);
+
+/*
  * fp4_quantize_noalloc -- fp4_quantize for NVFP4 / UFP4 with the tensor scale
  * taken from an internal amax, for callers that cannot allocate device
  * memory: code running where cudaMalloc is unavailable or forbidden (a plug-in

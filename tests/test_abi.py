@@ -194,3 +194,45 @@ def test_gemm_workspace_size():
     assert fp4.fp4_gemm_workspace_size(fp4.FP4_UFP4, False, 128, 128, 384) == 2 * (128 * 2 * 512 + 128 * 4 * 512 // 16)
     with pytest.raises(fp4.Fp4Error):
         fp4.fp4_gemm_workspace_size(9, False, 1, 1, 1)
+
+
+def oq(**kw):
+    a = dict(x=ADDR, dt=fp4.FP4_IN_BF16, rows=64, cols=256, ld=256, ch=ADDR, n=20, k8=128, rounding=0, rotation=0,
+             seed=0, tid=0, codes=ADDR, scales=ADDR, ts=ADDR, codes8=ADDR, s8=ADDR, ws=ADDR, wsb=4096)
+    a.update(kw)
+    return fp4._lib.fp4_outctl_quantize(a["x"], a["dt"], a["rows"], a["cols"], a["ld"], a["ch"], a["n"], a["k8"],
+                                        a["rounding"], a["rotation"], a["seed"], a["tid"], a["codes"], a["scales"],
+                                        a["ts"], a["codes8"], a["s8"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dt=2), 1), (dict(rounding=5), 1), (dict(n=-1), 1), (dict(n=200, k8=128), 1), (dict(ch=None), 1),
+    (dict(ts=None), 1), (dict(s8=None), 1), (dict(codes8=None), 1), (dict(codes=None), 1),
+    (dict(cols=248, ld=256), 2), (dict(k8=100), 2), (dict(rotation=2, cols=240, ld=256), 2),
+    (dict(codes8=ADDR + 8), 3), (dict(ch=ADDR + 2), 3), (dict(ws=ADDR + 4), 3),
+    (dict(ws=None), 4), (dict(wsb=100), 4),
+])
+def test_outctl_quantize_host_validation(kw, status):
+    assert oq(**kw) == status
+
+
+def og(**kw):
+    a = dict(a=ADDR, sa=ADDR, ta=ADDR, b=ADDR, sb=ADDR, tb=ADDR, a8=ADDR, s8a=ADDR, b8=ADDR, s8b=ADDR, M=256, N=256,
+             K=512, K8=128, c=ADDR, out=fp4.FP4_OUT_BF16, ldc=256)
+    a.update(kw)
+    return fp4._lib.fp4_gemm_outctl(a["a"], a["sa"], a["ta"], a["b"], a["sb"], a["tb"], a["a8"], a["s8a"], a["b8"],
+                                    a["s8b"], a["M"], a["N"], a["K"], a["K8"], a["c"], a["out"], a["ldc"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(out=2), 1), (dict(K8=-128), 1), (dict(ldc=100), 1), (dict(a8=None), 1), (dict(s8b=None), 1),
+    (dict(ta=None), 1), (dict(M=200), 2), (dict(K8=100), 2), (dict(K=0), 2), (dict(a8=ADDR + 8), 3),
+    (dict(c=ADDR + 4), 3),
+])
+def test_gemm_outctl_host_validation(kw, status):
+    assert og(**kw) == status
+
+
+def test_outctl_workspace_size():
+    assert fp4.fp4_outctl_workspace_size(4096) == 272 + 4096 // 8
+    assert fp4.fp4_outctl_workspace_size(0) == 272
