@@ -44,9 +44,9 @@ OPERANDS = workloads.LAYER_OPERANDS
 GEMMS = workloads.LAYER_GEMMS
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per gemm_kernel
 # launch, averaged over the 12 GEMM launches of one layer step, from one ncu
-# capture of the current kernel (profiles/gemm_layer_llama8b_t8192.md); None
-# until that capture exists
-GEMM_TRAFFIC_BYTES_PER_LAUNCH = None
+# capture of the current kernel (profiles/gemm_layer_llama8b_t8192.md); the
+# algorithmic bytes (operands read once, C written once) average 241.7 MB
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = 294_010_240
 
 
 class L2Flush:
@@ -391,7 +391,9 @@ def run_gpu(args, rank, world, device, host):
     # GEMM outputs) back.  Two sets of device buffers on three streams
     # (host->device, compute, device->host) let step i+1's inputs and step
     # i-1's results cross PCIe while step i computes.
-    e2e_steps = 4
+    e2e_steps = 0 if args.no_e2e else 4
+    if e2e_steps == 0:
+        return finish_line(args, rank, world, device, layer, fam, table, total_ms, None, 0, 0, clocks, status, peaks)
     hin = [{k: v.pin_memory() for k, v in h.items()} for h in host]
     hout = [[[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in lin["outs"]] for lin in layer.linears]
             for _ in range(2)]
@@ -439,7 +441,13 @@ def run_gpu(args, rank, world, device, host):
     del slots, second, hout
     torch.cuda.empty_cache()
 
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
+    return finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, h2d, d2h, clocks, status, peaks)
+
+
+def finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, h2d, d2h, clocks, status, peaks):
+    """Max over ranks of the timings, then rank 0's JSON line."""
+    from fp4_block_scaled_h16_b200 import fp4
+    t = torch.tensor([total_ms, e2e_ms if e2e_ms is not None else 0.0], dtype=torch.float64, device=device)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     total_max, e2e_max = float(t[0]), float(t[1])
@@ -456,6 +464,8 @@ def run_gpu(args, rank, world, device, host):
         roof = {"bound": "tensor", "kernel": "gemm_kernel (NVFP4, 12 launches per step)",
                 "achieved": round(f["tflops"], 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                 "frac": round(f["tflops"] / fp4_peak, 4), "traffic": GEMM_TRAFFIC_BYTES_PER_LAUNCH,
+                "traffic_is": "ncu DRAM read + write bytes per launch, averaged over the step's 12 GEMMs "
+                              "(algorithmic average 241.7 MB)",
                 "achieved_is": "GEMM FLOP of the step / summed mean event time of its 12 GEMM launches",
                 "peak_is": "%s bf16 burst %.1f TFLOP/s x 4 (nominal fp4 / bf16 ratio)" % (peaks["src"], peaks["bf16"])}
     else:
@@ -488,11 +498,12 @@ def run_gpu(args, rank, world, device, host):
                    "parallelism": "independent layer per GPU" if world > 1 else "single GPU"},
         "roofline": roof,
         "components": {"per_call": table},
-        "e2e": {"value": round(world * layer.flop / (e2e_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_max, 3),
-                "how": "fp4.quantize / fp4.gemm on the layer's inputs copied from pinned host memory every step, "
-                       "the 12 GEMM outputs copied back; two buffer sets on 3 streams overlap the copies of "
-                       "neighbouring steps with each other and with compute"},
+        "e2e": ({"value": round(world * layer.flop / (e2e_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_max, 3),
+                 "how": "fp4.quantize / fp4.gemm on the layer's inputs copied from pinned host memory every step, "
+                        "the 12 GEMM outputs copied back; two buffer sets on 3 streams overlap the copies of "
+                        "neighbouring steps with each other and with compute"}
+                if e2e_ms is not None else None),
         "gpu_launches": layer.launches * args.steps,
         "clocks": clocks.summary(),
         "device_status": fp4.fp4_status_string(status),
@@ -807,6 +818,8 @@ def main():
     ap.add_argument("--impl", choices=["fp4", "reference"], default="fp4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel table")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (host copies); for profiling the device step")
     ap.add_argument("--graph", action="store_true",
                     help="time the step replayed as one CUDA graph")
     ap.add_argument("--configs", default=",".join(CONFIG_NAMES),

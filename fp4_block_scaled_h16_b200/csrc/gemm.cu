@@ -88,14 +88,17 @@ __device__ __forceinline__ void raise_timeout(const GemmParams& p, volatile int*
 // for a half unit)
 template <int BN>
 __device__ __forceinline__ bool unit_geom(const GemmParams& p, int u, int& m0, int& n0) {
+    int tm, tn;
     if (u < p.split_base) {
-        m0 = (u % p.tiles_m) * BM;
-        n0 = (u / p.tiles_m) * BN;
+        tile_coords(u, p.tiles_m, p.tiles_n, tm, tn);
+        m0 = tm * BM;
+        n0 = tn * BN;
         return false;
     }
     const int t = p.split_base + ((u - p.split_base) >> 1);
-    m0 = (t % p.tiles_m) * BM;
-    n0 = (t / p.tiles_m) * BN + ((u - p.split_base) & 1) * (BN / 2);
+    tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+    m0 = tm * BM;
+    n0 = tn * BN + ((u - p.split_base) & 1) * (BN / 2);
     return true;
 }
 

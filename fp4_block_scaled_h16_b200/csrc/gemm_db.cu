@@ -134,7 +134,9 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             uint32_t phase = 0, fills = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN;
+                int tm_, tn_;
+                tile_coords(t, p.tiles_m, p.tiles_n, tm_, tn_);
+                const int m0 = tm_ * BM, n0 = tn_ * BN;
                 for (int kt = 0; kt < kt_count; ++kt) {
                     if (!sm100::mbar_wait(&empty[stage], phase ^ 1u, p.wait_limit, abort_flag)) {
                         raise_timeout(p, abort_flag);
@@ -225,7 +227,9 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         int ob = 0;
         uint32_t ophase = 0u;                         // bit b: phase of outer buffer b
         for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-            const int n0 = (t / p.tiles_m) * BN;
+            int tm_, tn_;
+            tile_coords(t, p.tiles_m, p.tiles_n, tm_, tn_);
+            const int n0 = tn_ * BN;
             int got = 0;
             if (lane == 0) got = sm100::mbar_wait(&oempty[ob], ((ophase >> ob) & 1u) ^ 1u, p.wait_limit, abort_flag) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, got, 0)) {
@@ -254,7 +258,9 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         uint32_t pphase = 0u, ophase = 0u;            // bit b: phase of buffer b
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN + cg * COLS;
+            int tm_, tn_;
+                tile_coords(t, p.tiles_m, p.tiles_n, tm_, tn_);
+                const int m0 = tm_ * BM, n0 = tn_ * BN + cg * COLS;
             const int row = m0 + 32 * q + lane;
             if (!__all_sync(0xffffffffu, sm100::mbar_wait(&ofull[ob], (ophase >> ob) & 1u, p.wait_limit, abort_flag))) {
                 if (lane == 0) raise_timeout(p, abort_flag);

@@ -114,7 +114,9 @@ gemm_outctl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             uint32_t phase = 0, fills = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN;
+                int tm_, tn_;
+                tile_coords(t, p.tiles_m, p.tiles_n, tm_, tn_);
+                const int m0 = tm_ * BM, n0 = tn_ * BN;
                 for (int kt = 0; kt < kt4 + kt8; ++kt) {
                     if (!sm100::mbar_wait(&empty[stage], phase ^ 1u, p.wait_limit, abort_flag)) {
                         raise_timeout(p, abort_flag);
@@ -217,7 +219,9 @@ gemm_outctl_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         const float a8 = p.K8 > 0 ? __fmul_rn(*p.a_s8, *p.b_s8) : 0.0f;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-            const int m0 = (t % p.tiles_m) * BM, n0 = (t / p.tiles_m) * BN + half * COLS;
+            int tm_, tn_;
+                tile_coords(t, p.tiles_m, p.tiles_n, tm_, tn_);
+                const int m0 = tm_ * BM, n0 = tn_ * BN + half * COLS;
             int got = 0;
             if (lane == 0) {
                 got = sm100::mbar_wait(acc_full, acc_phase, p.wait_limit, abort_flag) ? 1 : 0;

@@ -89,6 +89,21 @@ struct GemmArgs {
     uint32_t wait_limit;
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// Output tile t of a tiles_m x tiles_n grid in grouped order: bands of up to
+// GEMM_GROUP_M m-tiles, each band walked column by column.  The CTAs of one
+// persistent wave then share a compact block of A rows and B columns, so an
+// operand larger than L2 is read from DRAM about once instead of once per
+// column of tiles.
+constexpr int GEMM_GROUP_M = 8;
+__host__ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
+    const int band = t / (GEMM_GROUP_M * tiles_n);
+    const int first_m = band * GEMM_GROUP_M;
+    const int gm = (tiles_m - first_m) < GEMM_GROUP_M ? (tiles_m - first_m) : GEMM_GROUP_M;
+    const int local = t - band * GEMM_GROUP_M * tiles_n;
+    tm = first_m + local % gm;
+    tn = local / gm;
+}
 // OutControl (outctl.cu, gemm_outctl.cu)
 cudaError_t launch_channel_amax(const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld, float* out,
                                 cudaStream_t s);

@@ -44,11 +44,15 @@ enum ColMode { QC_QUANT = 0, QC_AMAX = 1, QC_FUSED = 2 };
 __device__ __forceinline__ uint32_t qc_ring_limit(uint32_t w) { return w >= (1u << 27) ? 0xFFFFFFFFu : w << 4; }
 __device__ __forceinline__ uint32_t qc_grid_limit(uint32_t w) { return w >= (1u << 29) ? 0xFFFFFFFFu : w << 2; }
 
-template <bool BF16>
+// Four CTAs per SM (128 registers).  (Measured on B200: a fifth CTA for the
+// stochastic-rounding variants, at 96 registers with two stages, was no
+// faster: they are bound by their instruction count, not by occupancy.)
+template <bool BF16, bool SR>
 struct ColRing {
     static constexpr int ES = BF16 ? 2 : 4;
     static constexpr int BYTES = QC_ROWS * QC_COLS * ES;        // one tile: 16 KB (bf16) / 32 KB (f32)
     static constexpr int STAGES = BF16 ? 3 : 2;
+    static constexpr int CTAS = 4;                              // the launch bound
     static constexpr int SMEM = STAGES * BYTES + 128 /*alignment*/ + STAGES * 16 /*barriers*/;
 };
 
@@ -103,12 +107,12 @@ __device__ __forceinline__ float col_of(const float2& p, int c) { return (c & 1)
 // ALIGN4 (stochastic rounding only): cols % 4 == 0, so the four columns of a
 // row are one Philox counter; otherwise they may straddle two
 template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE, bool ALIGN4 = true>
-__global__ void __launch_bounds__(QC_THREADS, 4)
+__global__ void __launch_bounds__(QC_THREADS, (ColRing<BF16, SR>::CTAS))
 quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, const ColTiles ct) {
     constexpr bool AMAX_ONLY = MODE == QC_AMAX, FUSED = MODE == QC_FUSED;
     static_assert(!FUSED || (FMT != MXFP4 && !DB), "only a tensor-scaled format has an amax pass");
     static_assert(!DB || (FMT == NVFP4 && MODE == QC_QUANT), "double block: NVFP4 quantize only");
-    using Ring = ColRing<BF16>;
+    using Ring = ColRing<BF16, SR>;
     constexpr int STAGES = Ring::STAGES, BYTES = Ring::BYTES;
     constexpr int BLK = (FMT == MXFP4) ? 32 : 16;
     extern __shared__ uint8_t qc_smem_raw[];
@@ -494,7 +498,7 @@ bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int6
 
 template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE, bool ALIGN4>
 cudaError_t launch_cols_k(const QuantArgs& a, cudaStream_t s) {
-    using Ring = ColRing<BF16>;
+    using Ring = ColRing<BF16, SR>;
     auto kernel = quant_cols_kernel<BF16, FMT, SR, ROT, SIGNS, DB, MODE, ALIGN4>;
     static PerDeviceOnce setup;
     static int resident_on[kOnceDevices];
