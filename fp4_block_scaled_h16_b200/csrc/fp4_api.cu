@@ -21,6 +21,7 @@ int g_arch_ok[kMaxDevices];               // 0 unknown, 1 sm_100, -1 other
 unsigned int* g_err_ptr[kMaxDevices];
 std::mutex g_mu;
 uint32_t g_wait_limit = 1u << 20;
+int g_gemm_pairs = 1;
 
 // Philox4x32-10 on the host, for the random-sign word and the round keys
 // (Salmon et al., SC'11: multipliers 0xD2511F53 / 0xCD9E8D57, Weyl key bumps
@@ -125,6 +126,8 @@ const char* fp4_status_string(fp4_status_t s) {
 }
 
 void fp4_set_wait_limit(uint32_t polls) { g_wait_limit = polls ? polls : (1u << 20); }
+
+void fp4_set_gemm_cta_pairs(int enable) { g_gemm_pairs = enable ? 1 : 0; }
 
 size_t fp4_scales_bytes(int64_t lines, int64_t K, fp4_format_t format) {
     if (lines <= 0 || K <= 0) return 0;
@@ -577,6 +580,7 @@ fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
         g.out_bf16 = out_dtype == FP4_OUT_BF16;
         g.fmt = FP4_NVFP4;
         g.db = 0;
+        g.pairs = g_gemm_pairs;
         g.wait_limit = g_wait_limit;
         if (launch_gemm(g, s) != cudaSuccess) return FP4_ERR_CUDA;
         return FP4_OK;
@@ -588,6 +592,7 @@ fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
     g.out_bf16 = out_dtype == FP4_OUT_BF16;
     g.fmt = format;
     g.db = double_block;
+    g.pairs = g_gemm_pairs;
     g.wait_limit = g_wait_limit;
     if (launch_gemm(g, s) != cudaSuccess) return FP4_ERR_CUDA;
     return FP4_OK;

@@ -425,6 +425,21 @@ bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over C [M, N] (row pitch ldc) for the epilogue's tiled stores: box =
+// 128 bytes of a row (64 bf16 or 32 fp32) x 32 rows, 128-byte swizzle
+bool make_c_map(CUtensorMap* m, void* c, bool bf16, int64_t M, int64_t N, int64_t ldc) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int64_t es = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(ldc * es)};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / es), 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, c, dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -440,6 +455,7 @@ bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int6
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     if (g.db) return launch_gemm_db(g, s);
+    if (g.pairs && gemm_pair_fits(g)) return launch_gemm_pair(g, s);
     const bool n256 = (g.N % 256) == 0;
     if (g.fmt == MXFP4) {
         if (n256) return g.out_bf16 ? run<MXFP4, 256, true>(g, s) : run<MXFP4, 256, false>(g, s);

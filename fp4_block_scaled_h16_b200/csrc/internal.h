@@ -5,6 +5,7 @@
 #include <mutex>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "fp4_device.cuh"
 
@@ -86,9 +87,13 @@ struct GemmArgs {
     int out_bf16;
     int fmt;
     int db;
+    int pairs;        // 1: 256 x 256 tiles on CTA pairs where the shape allows (gemm_pair.cu)
     uint32_t wait_limit;
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+// the CTA-pair GEMM (gemm_pair.cu): M and N multiples of 256, no double block
+bool gemm_pair_fits(const GemmArgs& g);
+cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s);
 
 // Output tile t of a tiles_m x tiles_n grid in grouped order: bands of up to
 // GEMM_GROUP_M m-tiles, each band walked column by column.  The CTAs of one
@@ -138,6 +143,10 @@ cudaError_t launch_ufp4_split(const uint8_t* codes, const uint8_t* scales, int64
 cudaError_t launch_gemm_db(const GemmArgs& g, cudaStream_t s);
 // 2-D TMA map over packed codes [rows, K/2] bytes: box 128 bytes x box_rows, 128-byte swizzle
 bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K, int box_rows);
+// 2-D map over C [M, N] for tiled stores: box 128 bytes x 32 rows, 128-byte swizzle
+bool make_c_map(CUtensorMap* m, void* c, bool bf16, int64_t M, int64_t N, int64_t ldc);
+// the driver's cuTensorMapEncodeTiled (null when the driver has none)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 
 // One-time setup per device (kernel attributes and occupancy are properties of
 // the kernel on one device): run() calls init once for the current device and

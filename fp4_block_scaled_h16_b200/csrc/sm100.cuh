@@ -1,7 +1,7 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the
-// GEMM uses: mbarriers with bounded waits, TMA tiled and bulk copies (never with
-// cluster multicast), tcgen05 TMEM allocation, smem->TMEM copies, block-scaled
-// MMAs, commits and TMEM loads.
+// GEMMs use: mbarriers with bounded waits, TMA tiled and bulk copies (never with
+// cluster multicast) and tiled stores, tcgen05 TMEM allocation, smem->TMEM
+// copies, block-scaled MMAs, commits and TMEM loads, and the CTA-pair forms.
 #pragma once
 
 #include <cstdint>
@@ -76,6 +76,24 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// tiled store shared -> global of one box (bulk async group of this thread)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's committed bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -161,14 +179,15 @@ __host__ __device__ constexpr uint32_t idesc_f8_e4m3(int n) {
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// instruction descriptor of the block-scaled MMA (M = 128, K = 64, both
-// operands E2M1 and K-major, FP32 accumulate)
-__host__ __device__ constexpr uint32_t idesc_block_scaled(int n, bool ue8m0, uint32_t a_sf_id, uint32_t b_sf_id) {
+// instruction descriptor of the block-scaled MMA (M = 128, or 256 over a CTA
+// pair; K = 64, both operands E2M1 and K-major, FP32 accumulate)
+__host__ __device__ constexpr uint32_t idesc_block_scaled(int n, bool ue8m0, uint32_t a_sf_id, uint32_t b_sf_id,
+                                                           int m = 128) {
     return (b_sf_id << 4)             // B scale-factor byte
          | (1u << 7) | (1u << 10)     // A, B format: E2M1
          | ((uint32_t)(n >> 3) << 17) // N / 8
          | ((ue8m0 ? 1u : 0u) << 23)  // scale format: 0 = UE4M3, 1 = UE8M0
-         | ((uint32_t)(128 >> 4) << 24)  // M / 16
+         | ((uint32_t)(m >> 4) << 24) // M / 16 (256 for a CTA pair)
          | (a_sf_id << 29);           // A scale-factor byte
 }
 
@@ -209,6 +228,121 @@ __device__ __forceinline__ void tmem_ld_wait_on(uint32_t (&r)[16]) {
                    "+r"(r[15])
                  :
                  : "memory");
+}
+
+// ------------------------------------------------------------------ CTA pairs
+// The pair GEMM runs on clusters of two CTAs: rank 0 (the leader) issues the
+// MMAs of cta_group::2 over both CTAs' shared memory and TMEM.  Every
+// tcgen05 instruction of such a kernel names cta_group::2.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// shared::cluster address of the object at the same offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+// every thread of both CTAs; orders shared-memory and barrier state across the pair
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// arrive on an mbarrier of either CTA (address from cluster_addr), release at cluster scope
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+
+// take `bytes` off the pending transaction count of a local mbarrier without arriving
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cluster.relaxed.cluster.b64 [%0], %1;"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
+    asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
+}
+
+// as mbar_wait, acquiring at cluster scope (arrivals from the peer CTA)
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t limit,
+                                                  const volatile int* abort_flag) {
+    for (uint32_t i = 0; i < limit; ++i) {
+        uint32_t ok;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+        if (ok) return true;
+        if ((i & 255u) == 255u && abort_flag && *abort_flag) return false;
+    }
+    return false;
+}
+
+// 2-D / 3-D tiled loads into this CTA's shared memory whose completion is
+// counted on the mbarrier at `bar_caddr` (the leader's, from cluster_addr);
+// no multicast
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                                 uint32_t bar_caddr) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_caddr)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                                 int32_t z, uint32_t bar_caddr) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_caddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// arrive on the mbarrier at this offset in both CTAs (mask 0b11) once the
+// pair's previously issued tcgen05 operations complete
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
+    asm volatile("{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+                 "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+// the same, on this CTA's mbarrier only
+__device__ __forceinline__ void tc_commit_pair_local(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+// scale-factor atom copy into both CTAs' TMEM, each from its own shared memory
+__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// M = 256 block-scaled MMAs over the pair: rows 0-127 of A and D in the
+// leader, 128-255 in the peer; B's first N / 2 rows from the leader's shared
+// memory, the rest from the peer's
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                 ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb) : "memory");
+}
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                 ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb) : "memory");
 }
 
 __device__ __forceinline__ bool elect_one() {

@@ -35,7 +35,7 @@ EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_q
            "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit",
            "fp4_quantize_noalloc", "fp4_requantize", "fp4_rotate", "fp4_mxnorm_quantize",
            "fp4_gemm_workspace_size", "fp4_channel_amax", "fp4_outctl_workspace_size", "fp4_outctl_quantize",
-           "fp4_gemm_outctl")
+           "fp4_gemm_outctl", "fp4_set_gemm_cta_pairs")
 
 _P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_uint32, ctypes.c_size_t)
@@ -63,6 +63,8 @@ _lib.fp4_gemm_workspace_size.argtypes = [_I, _I, _I64, _I64, _I64, ctypes.POINTE
 _lib.fp4_last_error.argtypes = [_P]
 _lib.fp4_set_wait_limit.argtypes = [_U32]
 _lib.fp4_set_wait_limit.restype = None
+_lib.fp4_set_gemm_cta_pairs.argtypes = [_I]
+_lib.fp4_set_gemm_cta_pairs.restype = None
 for _f in ("fp4_amax", "fp4_rotate", "fp4_mxnorm_quantize", "fp4_gemm_workspace_size", "fp4_channel_amax",
            "fp4_outctl_workspace_size", "fp4_outctl_quantize", "fp4_gemm_outctl", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
            "fp4_quantize_workspace_size"):
@@ -114,6 +116,10 @@ def fp4_quantize_workspace_size(fmt: int, double_block: bool, amax_given: bool) 
 
 def fp4_set_wait_limit(polls: int) -> None:
     _lib.fp4_set_wait_limit(polls)
+
+
+def fp4_set_gemm_cta_pairs(enable: bool) -> None:
+    _lib.fp4_set_gemm_cta_pairs(int(bool(enable)))
 
 
 def fp4_amax(x, in_dtype, rows, cols, ld, rotation, axis, seed, amax_out, stream=None) -> None:

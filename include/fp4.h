@@ -444,6 +444,17 @@ const char* fp4_status_string(fp4_status_t status);
  */
 void fp4_set_wait_limit(uint32_t polls);
 
+/*
+ * fp4_set_gemm_cta_pairs -- whether later fp4_gemm calls (MXFP4, NVFP4 and
+ * UFP4; not the double block) with M and N multiples of 256 run on CTA pairs:
+ * 256 x 256 output tiles shared by two SMs through tcgen05 cta_group::2, each
+ * SM loading its own A rows and half of B (nonzero, the default), or on single
+ * CTAs with 128 x 256 tiles (0).  The products are the same block-scaled dot
+ * products either way.  Process-wide; not synchronized with calls in flight on
+ * other host threads.
+ */
+void fp4_set_gemm_cta_pairs(int enable);
+
 #ifdef __cplusplus
 }
 #endif

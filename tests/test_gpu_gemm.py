@@ -34,11 +34,21 @@ def rand(M, K, seed, scale=1.0):
     return torch.from_numpy(x)
 
 
+@pytest.fixture(params=[True, False], ids=["pairs", "single"])
+def cta_pairs(fp4, request):
+    """Runs the test with 256 x 256 tiles on CTA pairs where M and N allow it
+    (the default), then with single-CTA 128 x 256 tiles only."""
+    fp4.fp4_set_gemm_cta_pairs(request.param)
+    yield request.param
+    fp4.fp4_set_gemm_cta_pairs(True)
+
+
 @pytest.mark.parametrize("out_bf16", [False, True])
 @pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 512), (384, 256, 1024), (128, 512, 2304),
-                                   (128, 256, 128), (256, 128, 384), (384, 512, 1152)])
-def test_gemm_on_oracle_operands(fp4, fmt, out_bf16, shape):
+                                   (128, 256, 128), (256, 128, 384), (384, 512, 1152),
+                                   (256, 256, 256), (512, 768, 1152), (256, 512, 128), (768, 256, 2048)])
+def test_gemm_on_oracle_operands(fp4, fmt, out_bf16, shape, cta_pairs):
     M, N, K = shape
     a, b = rand(M, K, M + K + fmt), rand(N, K, N + 3 * K + fmt, 0.1)
     qa = oracle_quantize(a, fmt=fmt, rotation=1)
@@ -53,10 +63,11 @@ def test_gemm_on_oracle_operands(fp4, fmt, out_bf16, shape):
 
 @pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("shape", [(5120, 1024, 256), (2560, 2048, 512), (5120, 1024, 384)])
-def test_gemm_with_more_tiles_than_sms_on_oracle_operands(fp4, fmt, shape):
-    # more 128x256 tiles than SMs (160 tiles on 148 SMs: a second, nearly
-    # empty wave of persistent tiles, run as 128-column halves; K = 384 ends
-    # on a half stage); every element against the oracle
+def test_gemm_with_more_tiles_than_sms_on_oracle_operands(fp4, fmt, shape, cta_pairs):
+    # single CTAs: more 128x256 tiles than SMs (160 tiles on 148 SMs: a
+    # second, nearly empty wave of persistent tiles, run as 128-column halves;
+    # K = 384 ends on a half stage).  CTA pairs: 80 256x256 tiles on 74 pairs,
+    # a second wave of 6.  Every element against the oracle.
     M, N, K = shape
     a, b = rand(M, K, M + fmt), rand(N, K, N + 7 + fmt, 0.1)
     qa = oracle_quantize(a, fmt=fmt)
@@ -66,6 +77,31 @@ def test_gemm_with_more_tiles_than_sms_on_oracle_operands(fp4, fmt, shape):
     torch.cuda.synchronize()
     assert fp4.fp4_last_error() == fp4.FP4_OK
     assert_within_gemm_bound(C.float().cpu().numpy(), C64, bound, True, what=str((fmt, shape)))
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("shape", [(512, 512, 1024), (2048, 1536, 640)])
+def test_pair_and_single_cta_tiles_give_the_same_bits(fp4, fmt, shape):
+    """The pair MMA (M = 256 over two SMs) and the single-CTA MMA (M = 128)
+    take the same 64-element K slices in the same order for every output, so
+    the two paths agree bit for bit; both stay within the oracle's bound."""
+    M, N, K = shape
+    a, b = rand(M, K, 3 * M + fmt), rand(N, K, 5 * N + fmt, 0.1)
+    qa, qb = oracle_quantize(a, fmt=fmt, rotation=1), oracle_quantize(b, fmt=fmt, rotation=1)
+    ta, tb = upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb)
+    out = {}
+    try:
+        for pairs in (True, False):
+            fp4.fp4_set_gemm_cta_pairs(pairs)
+            out[pairs] = fp4.gemm(ta, tb, fp4.FP4_OUT_F32)
+            torch.cuda.synchronize()
+            assert fp4.fp4_last_error() == fp4.FP4_OK
+    finally:
+        fp4.fp4_set_gemm_cta_pairs(True)
+    C64, bound = oracle.gemm(qa, qb)
+    for pairs in (True, False):
+        assert_within_gemm_bound(out[pairs].cpu().numpy(), C64, bound, False, what=str((fmt, shape, pairs)))
+    assert torch.equal(out[True].view(torch.int32), out[False].view(torch.int32))
 
 
 def test_gemm_ldc_larger_than_n(fp4):

@@ -34,27 +34,37 @@ def operands(fp4, fmt, double_block, M=256, N=256, K=8192, seed=5):
     return fp4.quantize(a, tensor_id=1, **kw), fp4.quantize(b, tensor_id=2, **kw)
 
 
-@pytest.mark.parametrize("fmt,double_block,out", [
-    ("MXFP4", False, "F32"),
-    ("NVFP4", False, "BF16"),
-    ("NVFP4", True, "BF16"),
-    ("NVFP4", True, "F32"),
+# (M, N) = (256, 256) runs on one CTA pair unless pairs are switched off, and
+# (512, 256) on two; the pair kernel's leader then also settles the loads
+# that only one of the two CTAs issued before it gave up.
+@pytest.mark.parametrize("fmt,double_block,out,pairs,M", [
+    ("MXFP4", False, "F32", True, 256),
+    ("NVFP4", False, "BF16", True, 256),
+    ("NVFP4", False, "F32", True, 512),
+    ("MXFP4", False, "F32", False, 256),
+    ("NVFP4", False, "BF16", False, 256),
+    ("NVFP4", True, "BF16", False, 256),
+    ("NVFP4", True, "F32", False, 256),
 ])
-def test_gemm_wait_timeout_is_reported_and_recoverable(fp4, fmt, double_block, out):
-    qa, qb = operands(fp4, getattr(fp4, "FP4_" + fmt), double_block)
+def test_gemm_wait_timeout_is_reported_and_recoverable(fp4, fmt, double_block, out, pairs, M):
+    qa, qb = operands(fp4, getattr(fp4, "FP4_" + fmt), double_block, M=M)
     out_dtype = getattr(fp4, "FP4_OUT_" + out)
-    before = fp4.gemm(qa, qb, out_dtype)
-    assert fp4.fp4_last_error() == fp4.FP4_OK
-
-    fp4.fp4_set_wait_limit(1)
+    fp4.fp4_set_gemm_cta_pairs(pairs)
     try:
-        fp4.gemm(qa, qb, out_dtype)
-        status = fp4.fp4_last_error()
-    finally:
-        fp4.fp4_set_wait_limit(0)
-    assert status == fp4.FP4_ERR_TIMEOUT, fp4.fp4_status_string(status)
+        before = fp4.gemm(qa, qb, out_dtype)
+        assert fp4.fp4_last_error() == fp4.FP4_OK
 
-    after = fp4.gemm(qa, qb, out_dtype)
+        fp4.fp4_set_wait_limit(1)
+        try:
+            fp4.gemm(qa, qb, out_dtype)
+            status = fp4.fp4_last_error()
+        finally:
+            fp4.fp4_set_wait_limit(0)
+        assert status == fp4.FP4_ERR_TIMEOUT, fp4.fp4_status_string(status)
+
+        after = fp4.gemm(qa, qb, out_dtype)
+    finally:
+        fp4.fp4_set_gemm_cta_pairs(True)
     assert fp4.fp4_last_error() == fp4.FP4_OK
     assert torch.equal(before.view(torch.int16 if out == "BF16" else torch.int32),
                        after.view(torch.int16 if out == "BF16" else torch.int32))
