@@ -42,11 +42,11 @@ T = workloads.TOKENS
 L2_FLUSH_BYTES = 256 << 20
 OPERANDS = workloads.LAYER_OPERANDS
 GEMMS = workloads.LAYER_GEMMS
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per gemm_kernel
-# launch, averaged over the 12 GEMM launches of one layer step, from one ncu
-# capture of the current kernel (profiles/gemm_layer_llama8b_t8192.md); the
-# algorithmic bytes (operands read once, C written once) average 241.7 MB
-GEMM_TRAFFIC_BYTES_PER_LAUNCH = 294_010_240
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per GEMM launch,
+# averaged over the 12 GEMM launches of one layer step, from one ncu capture of
+# the current kernel (profiles/gemm_layer_llama8b_t8192.md); the algorithmic
+# bytes (operands read once, C written once) average 241.7 MB
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = 276_410_112
 
 
 class L2Flush:
@@ -461,7 +461,7 @@ def finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, 
     dom = max(fam, key=lambda k: fam[k]["ms"])
     f = fam[dom]
     if dom == "gemm":
-        roof = {"bound": "tensor", "kernel": "gemm_kernel (NVFP4, 12 launches per step)",
+        roof = {"bound": "tensor", "kernel": "gemm_pair_kernel (NVFP4, 256x256 tiles on CTA pairs, 12 launches per step)",
                 "achieved": round(f["tflops"], 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                 "frac": round(f["tflops"] / fp4_peak, 4), "traffic": GEMM_TRAFFIC_BYTES_PER_LAUNCH,
                 "traffic_is": "ncu DRAM read + write bytes per launch, averaged over the step's 12 GEMMs "
