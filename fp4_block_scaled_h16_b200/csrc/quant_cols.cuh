@@ -61,31 +61,6 @@ struct ColTiles {
     uint32_t tc_m, tc_l;        // multiply-shift division by n_tc
 };
 
-// Stochastic rounding of |v| onto E2M1 with random word r: up from the level
-// below iff (r >> 8) * 2^-24 < (u - lo) / w, u = min(|v|, 6).  For u >= 1 the
-// levels are u's exponent with one mantissa bit: "up" is a carry out of the
-// 22 low mantissa bits when 2^22 - 1 - (r >> 10) is added to them (the test
-// (r >> 10) < m22, as 2^24 (u - lo) / w = 4 m22).  For u < 1 the bins are
-// [0, .5) and [.5, 1) of width 0.5: with X = ceil(2^25 u), the level index is
-// [r' < X] + [r' + 2^24 < X], r' = r >> 8.  Returns the magnitude index.
-__device__ __forceinline__ uint32_t sr_e2m1_col(float v, uint32_t r) {
-    const float u = fminf(fabsf(v), 6.0f);
-    const uint32_t ub = __float_as_uint(u);
-    const uint32_t hi = (ub + ((~r) >> 10) - (252u << 22)) >> 22;
-    const uint32_t X = __float2uint_ru(__fmul_rn(u, 0x1p25f));
-    const uint32_t rp = r >> 8;
-    const uint32_t lo = (rp < X ? 1u : 0u) + (rp + (1u << 24) < X ? 1u : 0u);
-    return u >= 1.0f ? hi : lo;
-}
-
-// the same on the uniform grid k = 0..7 (w = 1): up iff r' < ceil(2^24 (u - floor u))
-__device__ __forceinline__ uint32_t sr_ufp4_col(float v, uint32_t r) {
-    const float u = fminf(fabsf(v), 7.0f);
-    const float t = floorf(u);
-    const uint32_t F = __float2uint_ru(__fmul_rn(__fsub_rn(u, t), 0x1p24f));
-    return (uint32_t)t + ((r >> 8) < F ? 1u : 0u);
-}
-
 // 8 values of one column (rows 2i, 2i+1 in byte i) -> a word of E2M1 codes,
 // round to nearest even, saturating; a value that rounds to zero keeps its sign
 __device__ __forceinline__ uint32_t e2m1_rn8(float a0, float a1, float a2, float a3, float a4, float a5, float a6,
@@ -450,11 +425,14 @@ quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, co
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const float x = col_of(v[j + rr][c >> 1], c);
-                        uint32_t k;
-                        if (FMT == UFP4) k = SR ? sr_ufp4_col(x, rw[rr][c]) : (uint32_t)__float2int_rn(fminf(fabsf(x), 7.0f));
-                        else k = sr_e2m1_col(x, rw[rr][c]);
-                        const uint32_t nib = k | ((__float_as_uint(x) >> 28) & 8u);
-                        cw[c][(j + rr) >> 3] |= nib << (4 * ((j + rr) & 7));
+                        const int nb = (j + rr) & 7;
+                        if (FMT == UFP4 && !SR) {
+                            const uint32_t k = (uint32_t)__float2int_rn(fminf(fabsf(x), 7.0f));
+                            cw[c][(j + rr) >> 3] |= (k | ((__float_as_uint(x) >> 28) & 8u)) << (4 * nb);
+                        } else {
+                            cw[c][(j + rr) >> 3] |= sr_nibble(FMT == UFP4 ? sr_ufp4_sum(x, rw[rr][c])
+                                                                          : sr_e2m1_sum(x, rw[rr][c]), x, nb);
+                        }
                     }
                 }
             }

@@ -334,36 +334,37 @@ __device__ __forceinline__ void nv_divide(float* v, const float2* SY) {
 
 // ------------------------------------------------------------------ encoders
 
-// Stochastic rounding of |v| onto E2M1, as an exact integer test: with lo the
-// level below u = min(|v|, 6), w the gap above it and t = (r >> 8) * 2^-24,
-// "round up iff t < (u - lo) / w" is "(r >> 8) < ceil(2^24 (u - lo) / w)".
-// For u >= 1 the levels are u's exponent with one mantissa bit, so lo clears
-// the low 22 mantissa bits and 2^24 (u - lo) / w is those bits times 4; on
-// [0.5, 1) lo = 0.5, w = 0.5 and it is the 23-bit mantissa times 2; below
-// 0.5 it is u * 2^25.  Returns the magnitude index.
-__device__ __forceinline__ uint32_t sr_e2m1(float v, uint32_t r) {
+// Stochastic rounding of |v| onto E2M1 as one exact integer carry.  With lo
+// the level below u = min(|v|, 6), w the gap above it and t = (r >> 8) * 2^-24,
+// "round up iff t < (u - lo) / w" is "(r >> 8) < F", F = ceil(2^24 (u - lo) / w).
+// The levels are multiples of w = 0.5 on [0, 2), of 1 on [2, 4) and of 2 on
+// [4, 6], so with X = ceil(2^25 u) (exact: 2^25 u is an integer unless u <
+// 1/4, and then only the ceiling matters) and s = 0, 1, 2 the binade shift,
+// Y = X >> s holds the index of lo within its binade above bit 24 and F in its
+// low 24 bits.  Adding 2^24 - 1 - (r >> 8) = (~r) >> 8 carries into bit 24
+// exactly when (r >> 8) < F; adding s << 25 turns the binade's first index (0,
+// 2, 2) into the code's (0, 4, 6).  Returns the sum: the magnitude index in
+// bits 24-26, zeros above (the sum stays below 2^27).
+__device__ __forceinline__ uint32_t sr_e2m1_sum(float v, uint32_t r) {
     const float u = fminf(fabsf(v), 6.0f);
-    const uint32_t ub = __float_as_uint(u);
-    uint32_t lo_idx, F;
-    if (u >= 1.0f) {
-        lo_idx = (ub >> 22) - 252u;                // 1 -> 2, 1.5 -> 3, 2 -> 4, ... 6 -> 7
-        F = (ub & 0x3FFFFFu) << 2;
-    } else if (u >= 0.5f) {
-        lo_idx = 1u;
-        F = (ub & 0x7FFFFFu) << 1;
-    } else {
-        lo_idx = 0u;
-        F = __float2uint_ru(__fmul_rn(u, 0x1p25f));
-    }
-    return lo_idx + ((r >> 8) < F ? 1u : 0u);
+    const uint32_t X = __float2uint_ru(__fmul_rn(u, 0x1p25f));
+    const uint32_t s = min(X >> 26, 2u);
+    return (X >> s) + ((~r) >> 8) + (s << 25);
 }
 
-// the same on the uniform grid k = 0..7: lo = floor(u), w = 1
-__device__ __forceinline__ uint32_t sr_ufp4(float v, uint32_t r) {
+// the same on the uniform grid k = 0..7 (w = 1): X = ceil(2^24 u) holds floor(u)
+// above bit 24 and F below it
+__device__ __forceinline__ uint32_t sr_ufp4_sum(float v, uint32_t r) {
     const float u = fminf(fabsf(v), 7.0f);
-    const float t = floorf(u);
-    const uint32_t F = __float2uint_ru(__fmul_rn(__fsub_rn(u, t), 0x1p24f));
-    return (uint32_t)t + ((r >> 8) < F ? 1u : 0u);
+    return __float2uint_ru(__fmul_rn(u, 0x1p24f)) + ((~r) >> 8);
+}
+
+// nibble j (0..7, a compile-time constant after unrolling) of a code word from
+// such a sum and the sign bit of the value: magnitude bits from bits 24-26 of
+// the sum, sign from bit 31 of x
+__device__ __forceinline__ uint32_t sr_nibble(uint32_t sum, float x, int j) {
+    const uint32_t mag = (j < 7) ? (sum >> (24 - 4 * j)) : (sum << 4);
+    return (mag & (7u << (4 * j))) | ((__float_as_uint(x) >> (28 - 4 * j)) & (8u << (4 * j)));
 }
 
 // 8 scaled values -> one word of codes, element j in nibble j
@@ -386,11 +387,13 @@ __device__ __forceinline__ uint32_t encode8(const float* v, const uint32_t* rnd)
     uint32_t w = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        uint32_t k;
-        if (FMT == UFP4) k = SR ? sr_ufp4(v[j], rnd[j]) : (uint32_t)__float2int_rn(fminf(fabsf(v[j]), 7.0f));
-        else             k = sr_e2m1(v[j], rnd[j]);
-        // magnitude and sign bit (bit 31 of v moved to bit 3 of the nibble)
-        w |= (k | ((__float_as_uint(v[j]) >> 28) & 8u)) << (4 * j);
+        if (FMT == UFP4 && !SR) {
+            // magnitude and sign bit (bit 31 of v moved to bit 3 of the nibble)
+            const uint32_t k = (uint32_t)__float2int_rn(fminf(fabsf(v[j]), 7.0f));
+            w |= (k | ((__float_as_uint(v[j]) >> 28) & 8u)) << (4 * j);
+        } else {
+            w |= sr_nibble(FMT == UFP4 ? sr_ufp4_sum(v[j], rnd[j]) : sr_e2m1_sum(v[j], rnd[j]), v[j], j);
+        }
     }
     return w;
 }
