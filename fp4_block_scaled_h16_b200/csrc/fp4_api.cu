@@ -543,7 +543,6 @@ fp4_status_t fp4_gemm(fp4_format_t format, int double_block,
     if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return FP4_OK;
     if (M % 128 || N % 128 || K % 128 || K == 0) return FP4_ERR_UNSUPPORTED_SHAPE;
-    if (double_block && K > 8192) return FP4_ERR_UNSUPPORTED_SHAPE;
     if (!a_codes || !a_scales || !b_codes || !b_scales || !c) return FP4_ERR_INVALID_ARG;
     if (format != FP4_MXFP4 && !double_block && (!a_tensor_scale || !b_tensor_scale)) return FP4_ERR_INVALID_ARG;
     if (double_block && (!a_outer || !b_outer)) return FP4_ERR_INVALID_ARG;

@@ -8,15 +8,16 @@
 // The outer scale changes every 128 elements of K, so it cannot ride in the
 // tensor core's E4M3 block scales.  Each 128-K chunk is two block-scaled MMAs
 // (tcgen05 kind::mxf4nvf4, 128 x 128 x 64) into one of three TMEM partial
-// buffers in rotation; while the tensor core fills one, sixteen epilogue
-// warps (four per TMEM lane quarter, so each scheduler has four to hide the
-// TMEM and shared-load latency) promote another:
+// buffers in rotation; while the tensor core fills one, eight epilogue warps
+// (two per TMEM lane quarter, 64 columns each, so that the per-chunk barrier
+// and bookkeeping work is shared by twice the arithmetic) promote another:
 // acc[i, j] += s_oA[i, kc] * (s_oB[j, kc] * P_kc[i, j]) in registers, on
 // packed f32x2 pairs.  The operand pipeline (TMA producer warp, MMA warp,
 // 4-stage ring of 256-K stages) is the one of the plain GEMM; one more warp
-// stages each tile's B outer scales transposed ([chunk][column]) into a
-// double-buffered shared area, so the promotion reads four of them per
-// 128-bit shared load.  All hand-offs are mbarriers with bounded waits.
+// stages each tile's B outer scales transposed ([chunk][column]), in groups
+// of 64 chunks (any K), into a double-buffered shared area, so the promotion
+// reads four of them per 128-bit shared load.  All hand-offs are mbarriers
+// with bounded waits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -32,7 +33,7 @@ namespace {
 
 constexpr int BM = 128, BN = 128, BK = 256;
 constexpr int STAGES = 4;
-constexpr int EPI_WARPS = 16;             // four per TMEM lane quarter, a quarter of the columns each
+constexpr int EPI_WARPS = 8;              // two per TMEM lane quarter, half the columns each
 constexpr int COLS = BN / (EPI_WARPS / 4);      // columns one epilogue warp promotes
 constexpr int HALF = COLS / 2;                  // columns per TMEM load
 constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS + 1);   // producer, MMA, epilogue, outer-scale warp
@@ -40,13 +41,13 @@ constexpr int STAGER_WARP = 2 + EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t DRAIN_LIMIT = 1u << 22;
 constexpr unsigned int ERR_TIMEOUT = 7u;
-constexpr int MAX_CHUNKS = 64;                        // K / 128 <= 64: K <= 8192
+constexpr int MAX_CHUNKS = 64;                        // chunks of B outer scales per staged group
 
 constexpr uint32_t A_BYTES = BM * BK / 2, B_BYTES = BN * BK / 2;
 constexpr uint32_t SFA_BYTES = BM * (BK / 16), SFB_BYTES = BN * (BK / 16);
 constexpr uint32_t TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr uint32_t STAGE_BYTES = (TX + 1023) / 1024 * 1024;
-constexpr uint32_t OUTER_BYTES = 2 * MAX_CHUNKS * BN * 4;   // s_oB of two tiles, [chunk][column]
+constexpr uint32_t OUTER_BYTES = 2 * MAX_CHUNKS * BN * 4;   // two groups of s_oB, [chunk][column]
 constexpr uint32_t SMEM = STAGES * STAGE_BYTES + OUTER_BYTES + 1024 + 256;
 constexpr int PBUF = 3;                               // TMEM partial buffers in rotation
 constexpr uint32_t SFA_COL = PBUF * BN;               // TMEM: partials at 0, BN, 2 BN, then scales
@@ -230,25 +231,33 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             int tm_, tn_;
             tile_coords(t, p.tiles_m, p.tiles_n, tm_, tn_);
             const int n0 = tn_ * BN;
-            int got = 0;
-            if (lane == 0) got = sm100::mbar_wait(&oempty[ob], ((ophase >> ob) & 1u) ^ 1u, p.wait_limit, abort_flag) ? 1 : 0;
-            if (!__shfl_sync(0xffffffffu, got, 0)) {
-                if (lane == 0) raise_timeout(p, abort_flag);
-                break;
+            // the tile's B outer scales in groups of up to MAX_CHUNKS chunks,
+            // one group per buffer: rows n0 .. n0+127 of [N, K/128] written
+            // transposed ([chunk][column]); consecutive lanes take consecutive
+            // columns so the shared stores do not collide on a bank
+            bool staged = true;
+            for (int g0 = 0; g0 < nkc; g0 += MAX_CHUNKS) {
+                const int cnt = min(MAX_CHUNKS, nkc - g0);
+                int got = 0;
+                if (lane == 0)
+                    got = sm100::mbar_wait(&oempty[ob], ((ophase >> ob) & 1u) ^ 1u, p.wait_limit, abort_flag) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    if (lane == 0) raise_timeout(p, abort_flag);
+                    staged = false;
+                    break;
+                }
+                float* dst = outer_b + ob * (MAX_CHUNKS * BN);
+                const float* src = p.b_outer + (int64_t)n0 * nkc + g0;
+                for (int e = lane; e < BN * cnt; e += 32) {
+                    const int kc = e / BN, c = e % BN;
+                    dst[e] = __ldg(src + (int64_t)c * nkc + kc);
+                }
+                __syncwarp();
+                sm100::mbar_arrive(&ofull[ob]);          // release: every lane's stores before
+                ophase ^= 1u << ob;
+                ob ^= 1;
             }
-            // rows n0 .. n0+127 of [N, K/128] (16 KB at most, L1-resident after
-            // the first chunk) written transposed; consecutive lanes take
-            // consecutive columns so the shared stores do not collide on a bank
-            float* dst = outer_b + ob * (MAX_CHUNKS * BN);
-            const float* src = p.b_outer + (int64_t)n0 * nkc;
-            for (int e = lane; e < BN * nkc; e += 32) {
-                const int kc = e / BN, c = e % BN;
-                dst[e] = __ldg(src + c * nkc + kc);
-            }
-            __syncwarp();
-            sm100::mbar_arrive(&ofull[ob]);          // release: every lane's stores before
-            ophase ^= 1u << ob;
-            ob ^= 1;
+            if (!staged) break;
         }
     } else {
         // ------------------------------------------------------------ promotion + epilogue
@@ -262,11 +271,7 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 tile_coords(t, p.tiles_m, p.tiles_n, tm_, tn_);
                 const int m0 = tm_ * BM, n0 = tn_ * BN + cg * COLS;
             const int row = m0 + 32 * q + lane;
-            if (!__all_sync(0xffffffffu, sm100::mbar_wait(&ofull[ob], (ophase >> ob) & 1u, p.wait_limit, abort_flag))) {
-                if (lane == 0) raise_timeout(p, abort_flag);
-                break;
-            }
-            const float* outer_tile = outer_b + ob * (MAX_CHUNKS * BN) + cg * COLS;
+            const float* outer_tile = outer_b + cg * COLS;     // set per group of chunks below
             float2 acc[COLS / 2];
 #pragma unroll
             for (int c = 0; c < COLS / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
@@ -293,70 +298,81 @@ gemm_db_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 ok = false;
             } else {
                 sm100::tc_fence_after();
-                sm100::tmem_ld16(tbase + BN * pb, ra);
+                sm100::tmem_ld32(tbase + BN * pb, ra);
                 sm100::tmem_ld_wait_on(ra);
             }
-            for (int kc = 0; kc < nkc && ok; ++kc) {
-                const float sa = PAIRED ? ((kc & 1) ? sa_cur.y : sa_cur.x) : sa0;
-                const float2 sa2 = make_float2(sa, sa);
-                const float4* sb = reinterpret_cast<const float4*>(outer_tile + kc * BN);
-                sm100::tmem_ld16(tbase + BN * pb + HALF, rb);
-                // acc += sa * (sB * P) on the first half, packed
+            int kc = 0;
+            for (int g0 = 0; g0 < nkc && ok; g0 += MAX_CHUNKS) {
+                // the next group of B outer scales (chunks g0 .. gend - 1)
+                const int gend = min(nkc, g0 + MAX_CHUNKS);
+                if (!__all_sync(0xffffffffu, sm100::mbar_wait(&ofull[ob], (ophase >> ob) & 1u, p.wait_limit, abort_flag))) {
+                    if (lane == 0) raise_timeout(p, abort_flag);
+                    ok = false;
+                    break;
+                }
+                outer_tile = outer_b + ob * (MAX_CHUNKS * BN) + cg * COLS - g0 * BN;
+                for (; kc < gend && ok; ++kc) {
+                    const float sa = PAIRED ? ((kc & 1) ? sa_cur.y : sa_cur.x) : sa0;
+                    const float2 sa2 = make_float2(sa, sa);
+                    const float4* sb = reinterpret_cast<const float4*>(outer_tile + kc * BN);
+                    sm100::tmem_ld32(tbase + BN * pb + HALF, rb);
+                    // acc += sa * (sB * P) on the first half, packed
 #pragma unroll
-                for (int c = 0; c < HALF / 4; ++c) {
-                    const float4 w = sb[c];
-                    const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(ra[4 * c]), __uint_as_float(ra[4 * c + 1])),
-                                                 make_float2(w.x, w.y));
-                    const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(ra[4 * c + 2]), __uint_as_float(ra[4 * c + 3])),
-                                                 make_float2(w.z, w.w));
-                    acc[2 * c] = __ffma2_rn(t0, sa2, acc[2 * c]);
-                    acc[2 * c + 1] = __ffma2_rn(t1, sa2, acc[2 * c + 1]);
-                }
-                sm100::tmem_ld_wait_on(rb);
-                sm100::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) sm100::mbar_arrive(&pempty[pb]);     // the tensor core may refill it
-                pphase ^= 1u << pb;
-                pb = (pb + 1 == PBUF) ? 0 : pb + 1;
-                if (PAIRED) {
-                    if (kc & 1) {
-                        sa_cur = sa_nxt;
-                        if (kc + 3 < nkc) sa_nxt = __ldg(a_outer_pairs + (kc + 3) / 2);
+                    for (int c = 0; c < HALF / 4; ++c) {
+                        const float4 w = sb[c];
+                        const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(ra[4 * c]), __uint_as_float(ra[4 * c + 1])),
+                                                     make_float2(w.x, w.y));
+                        const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(ra[4 * c + 2]), __uint_as_float(ra[4 * c + 3])),
+                                                     make_float2(w.z, w.w));
+                        acc[2 * c] = __ffma2_rn(t0, sa2, acc[2 * c]);
+                        acc[2 * c + 1] = __ffma2_rn(t1, sa2, acc[2 * c + 1]);
                     }
-                } else {
-                    sa0 = sa1;
-                    sa1 = sa2n;
-                    if (kc + 3 < nkc) sa2n = __ldg(a_outer_row + kc + 3);
-                }
-                bool next = false;
-                if (kc + 1 < nkc) {
-                    if (__all_sync(0xffffffffu,
-                                   sm100::mbar_wait(&pfull[pb], (pphase >> pb) & 1u, p.wait_limit, abort_flag))) {
-                        sm100::tc_fence_after();
-                        sm100::tmem_ld16(tbase + BN * pb, ra);
-                        next = true;
+                    sm100::tmem_ld_wait_on(rb);
+                    sm100::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) sm100::mbar_arrive(&pempty[pb]);     // the tensor core may refill it
+                    pphase ^= 1u << pb;
+                    pb = (pb + 1 == PBUF) ? 0 : pb + 1;
+                    if (PAIRED) {
+                        if (kc & 1) {
+                            sa_cur = sa_nxt;
+                            if (kc + 3 < nkc) sa_nxt = __ldg(a_outer_pairs + (kc + 3) / 2);
+                        }
                     } else {
-                        if (lane == 0) raise_timeout(p, abort_flag);
-                        ok = false;
+                        sa0 = sa1;
+                        sa1 = sa2n;
+                        if (kc + 3 < nkc) sa2n = __ldg(a_outer_row + kc + 3);
                     }
-                }
-                // the second half, while the next chunk's first half loads
+                    bool next = false;
+                    if (kc + 1 < nkc) {
+                        if (__all_sync(0xffffffffu,
+                                       sm100::mbar_wait(&pfull[pb], (pphase >> pb) & 1u, p.wait_limit, abort_flag))) {
+                            sm100::tc_fence_after();
+                            sm100::tmem_ld32(tbase + BN * pb, ra);
+                            next = true;
+                        } else {
+                            if (lane == 0) raise_timeout(p, abort_flag);
+                            ok = false;
+                        }
+                    }
+                    // the second half, while the next chunk's first half loads
 #pragma unroll
-                for (int c = 0; c < HALF / 4; ++c) {
-                    const float4 w = sb[HALF / 4 + c];
-                    const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(rb[4 * c]), __uint_as_float(rb[4 * c + 1])),
-                                                 make_float2(w.x, w.y));
-                    const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(rb[4 * c + 2]), __uint_as_float(rb[4 * c + 3])),
-                                                 make_float2(w.z, w.w));
-                    acc[HALF / 2 + 2 * c] = __ffma2_rn(t0, sa2, acc[HALF / 2 + 2 * c]);
-                    acc[HALF / 2 + 2 * c + 1] = __ffma2_rn(t1, sa2, acc[HALF / 2 + 2 * c + 1]);
+                    for (int c = 0; c < HALF / 4; ++c) {
+                        const float4 w = sb[HALF / 4 + c];
+                        const float2 t0 = __fmul2_rn(make_float2(__uint_as_float(rb[4 * c]), __uint_as_float(rb[4 * c + 1])),
+                                                     make_float2(w.x, w.y));
+                        const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(rb[4 * c + 2]), __uint_as_float(rb[4 * c + 3])),
+                                                     make_float2(w.z, w.w));
+                        acc[HALF / 2 + 2 * c] = __ffma2_rn(t0, sa2, acc[HALF / 2 + 2 * c]);
+                        acc[HALF / 2 + 2 * c + 1] = __ffma2_rn(t1, sa2, acc[HALF / 2 + 2 * c + 1]);
+                    }
+                    if (next) sm100::tmem_ld_wait_on(ra);
                 }
-                if (next) sm100::tmem_ld_wait_on(ra);
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(&oempty[ob]);          // this group's outer scales are used
+                ophase ^= 1u << ob;
+                ob ^= 1;
             }
-            __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(&oempty[ob]);          // this tile's outer scales are used
-            ophase ^= 1u << ob;
-            ob ^= 1;
             if (!ok) break;
             // store this warp's part of the tile's row
             if (OUT_BF16) {
@@ -423,7 +439,6 @@ cudaError_t run_db(const GemmArgs& g, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_gemm_db(const GemmArgs& g, cudaStream_t s) {
-    if (g.K / 128 > MAX_CHUNKS) return cudaErrorInvalidValue;
     if ((g.K / 128) % 2 == 0) return g.out_bf16 ? run_db<true, true>(g, s) : run_db<false, true>(g, s);
     return g.out_bf16 ? run_db<true, false>(g, s) : run_db<false, false>(g, s);
 }

@@ -407,8 +407,7 @@ fp4_status_t fp4_gemm_workspace_size(fp4_format_t format, int double_block, int6
  *   c         device, [M, ldc] row-major, fp32 or bf16, ldc >= N
  *   workspace device, >= fp4_gemm_workspace_size() bytes, 16-byte aligned
  *             (UFP4 only; NULL and 0 otherwise); contents are scratch
- * Shape rules: M % 128 == 0, N % 128 == 0, K % 128 == 0 (double block: also
- * K <= 8192); ldc * size % 16 == 0.
+ * Shape rules: M % 128 == 0, N % 128 == 0, K % 128 == 0; ldc * size % 16 == 0.
  * The accumulation is FP32 on the tensor cores.
  */
 fp4_status_t fp4_gemm(fp4_format_t format, int double_block,

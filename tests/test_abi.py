@@ -99,7 +99,7 @@ UFP4_WS = 2 * (256 * 2 * 512 + 256 * 4 * 512 // 16)     # both operands' split c
     (dict(M=200), 2), (dict(N=192), 2), (dict(K=320), 2), (dict(K=0), 2),
     (dict(a=ADDR + 8), 3), (dict(ldc=260), 3),
     (dict(db=1, oa=ADDR + 8, ob=ADDR), 3), (dict(db=1, oa=ADDR, ob=ADDR + 4), 3),
-    (dict(db=1, oa=None, ob=ADDR), 1), (dict(db=1, K=8448, oa=ADDR, ob=ADDR), 2),
+    (dict(db=1, oa=None, ob=ADDR), 1),
 ])
 def test_gemm_host_validation(kw, status):
     assert g(**kw) == status

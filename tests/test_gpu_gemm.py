@@ -181,13 +181,18 @@ def test_full_mxfp4_wgrad_down(fp4):
 
 @pytest.mark.parametrize("out_bf16", [False, True])
 @pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 512), (128, 256, 2048), (384, 128, 8192),
-                                   (128, 128, 128), (256, 128, 384), (128, 256, 1152), (128, 128, 8064)])
+                                   (128, 128, 128), (256, 128, 384), (128, 256, 1152), (128, 128, 8064),
+                                   (128, 128, 8320), (256, 128, 16384), (128, 256, 24704)])
 def test_double_block_gemm_on_oracle_operands(fp4, out_bf16, shape):
-    """C = sum over 128-K chunks of s_oA * s_oB * (block-scaled partial)."""
+    """C = sum over 128-K chunks of s_oA * s_oB * (block-scaled partial).  K
+    past 8192 takes B's outer scales in several staged groups of 64 chunks
+    (8320: 64 + 1, 16384: 64 + 64, 24704: 3 x 64 + 1)."""
     M, N, K = shape
     a, b = rand(M, K, M + K), rand(N, K, 7 * N + K, 0.1)
-    # chunk magnitudes that vary along K, so every chunk's outer scale matters
+    # chunk magnitudes that vary along K on both operands, so every chunk's
+    # outer scales matter (and a group taken for the wrong chunks shows)
     a = a * torch.from_numpy(np.repeat(np.exp2(np.random.default_rng(1).integers(-6, 6, K // 128)), 128)).float()
+    b = b * torch.from_numpy(np.repeat(np.exp2(np.random.default_rng(2).integers(-6, 6, K // 128)), 128)).float()
     qa = oracle_quantize(a, fmt=NV, double_block=True, rounding=1, seed=3, tensor_id=1)
     qb = oracle_quantize(b, fmt=NV, double_block=True, rounding=1, seed=3, tensor_id=2)
     C64, bound = oracle.gemm(qa, qb)
@@ -209,9 +214,13 @@ def test_full_nvfp4_dgrad_double_block(fp4):
     sampled_gemm_check(fp4, qa, qb, d["dY"], d["Wd"], ka, kb, True, 96, 2)
 
 
-def test_double_block_gemm_rejects_long_k(fp4):
-    a = rand(128, 8448, 1)
-    qa = fp4.quantize(a.cuda(), fmt=NV, double_block=True)
-    with pytest.raises(fp4.Fp4Error) as e:
-        fp4.gemm(qa, qa)
-    assert e.value.status == fp4.FP4_ERR_UNSUPPORTED_SHAPE
+def test_double_block_gemm_long_k_whole_path(fp4):
+    """The double-block GEMM at K = 28672 (the gate+up Dgrad's contraction) on
+    GPU-quantized operands, sampled rows and columns against the oracle."""
+    M, N, K = 256, 512, 28672
+    a, b = rand(M, K, 11), rand(N, K, 12, 0.1)
+    ka = dict(fmt=NV, rounding=1, rotation=0, axis=1, double_block=True, seed=0, tensor_id=1)
+    kb = dict(fmt=NV, rounding=1, rotation=0, axis=1, double_block=True, seed=0, tensor_id=2)
+    qa = fp4.quantize(a.bfloat16().cuda(), **ka)
+    qb = fp4.quantize(b.bfloat16().cuda(), **kb)
+    sampled_gemm_check(fp4, qa, qb, a.bfloat16(), b.bfloat16(), ka, kb, True, 64, 3)
