@@ -59,7 +59,11 @@ def make(R, ld, dtype, seed):
 @pytest.mark.parametrize("rounding", [0, 1])
 @pytest.mark.parametrize("p", [1, 2])
 @pytest.mark.parametrize("fmt", [MX, NV, UF])
-@pytest.mark.parametrize("shape", [(37, 4096, 4096), (5, 14336, 14336), (130, 96, 128), (64, 4128, 4160)])
+# bf16 rows of 256 .. 4096 columns (a multiple of 256) run one warp per row
+# (11 and 5 chunks of 256: chunk sums padded to a power of two; a row pitch
+# wider than the row); the other shapes and f32 take the CTA-per-row kernel
+@pytest.mark.parametrize("shape", [(37, 4096, 4096), (5, 14336, 14336), (130, 96, 128), (64, 4128, 4160),
+                                   (300, 2816, 2816), (70, 256, 264), (9, 1280, 1280)])
 def test_mxnorm_matches_oracle(fp4, fmt, p, rounding, dtype, shape):
     R, C, ld = shape
     if C % (32 if fmt == MX else 16):
@@ -71,9 +75,10 @@ def test_mxnorm_matches_oracle(fp4, fmt, p, rounding, dtype, shape):
     compare(fp4, q, o, what=str((fmt, p, rounding, dtype, shape)))
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("p", [1, 2])
-def test_mxnorm_special_rows(fp4, fmt, p):
+def test_mxnorm_special_rows(fp4, fmt, p, dtype):
     rng = np.random.default_rng(2)
     x = rng.standard_normal((8, 512)).astype(np.float32)
     x[0] = 0.0                       # all zero: rho = 1
@@ -86,9 +91,11 @@ def test_mxnorm_special_rows(fp4, fmt, p):
     x[5, ::2] = 0.0
     c = c_of(p, fmt)
     xt = torch.from_numpy(x)
+    if dtype == "bf16":
+        xt = xt.to(torch.bfloat16)       # the subnormal row becomes zeros; 512 columns: the warp-per-row kernel
     q = fp4.mxnorm_quantize(xt.cuda(), fmt, p, c)
-    o = oracle.mxnorm(x, fmt, p, c)
-    compare(fp4, q, o, what="special %s" % ((fmt, p),))
+    o = oracle.mxnorm(oracle_input(xt), fmt, p, c)
+    compare(fp4, q, o, what="special %s" % ((fmt, p, dtype),))
     assert o["rho"][0] == 1.0
 
 
