@@ -17,7 +17,7 @@
 // max_t RN(rowmax_t * rho_t)) and then the quantize pass, which reads rho back.
 //
 // bf16 rows of up to 4096 columns (a multiple of 256) run one warp per row
-// with the row in registers (mxnorm_warp_kernel); other rows one CTA of 128
+// (mxnorm_warp_kernel); other rows one CTA of 128
 // threads per row at a time (grid-stride over the rows): the row is staged
 // in shared memory once, each thread takes blocks tid, tid + 128, ... for the
 // maxima and again for the cast.
@@ -210,17 +210,20 @@ mxnorm_kernel(const MxNormArgs a) {
 
 // ---------------------------------------------------------------- warp per row
 // bf16 rows of at most MNW_MAX_CHUNKS * 256 columns (a multiple of 256): one
-// warp per row, the row held in registers.  Chunk i (256 elements) gives lane
-// l the 8 elements [256 i + 8 l, 256 i + 8 l + 8) as one 16-byte word, so a
-// block is 2 lanes (16 elements) or 4 lanes (32).  Block maxima come from a
-// shuffle within the block's lanes.  The pairwise binary64 sum runs as a
-// butterfly inside each chunk, where every lane adds the same two subtrees
-// and so holds the chunk's subtree sum, then over the chunks in registers,
-// padded with zeros to a power of two: the same tree, node for node, as the
-// CTA kernel's, with no barrier.  The cast uses max |y| = RN(max |x| * rho)
-// per block (rounding is monotone) and writes each lane's 4 code bytes.
+// warp per row.  Chunk i (256 elements) gives lane l the 8 elements
+// [256 i + 8 l, 256 i + 8 l + 8) as one 16-byte word, so a block is 2 lanes
+// (16 elements) or 4 lanes (32), and its maximum comes from a shuffle within
+// them.  The pairwise binary64 sum runs as a butterfly inside each chunk,
+// where every lane adds the same two subtrees and so holds the chunk's
+// subtree sum; lane i keeps chunk i's, and a butterfly over lanes 0-15
+// (zeros past the last chunk) adds the chunks: the same tree, node for node,
+// as the CTA kernel's zero-padded one, with no barrier.  The row is read
+// twice, for the statistics and for the cast (the second read from L1/L2),
+// so that few registers leave room for many warps; the cast uses the block
+// maxima of the first read, max |y| = RN(max |x| * rho) (rounding is monotone).
 constexpr int MNW_WARPS = 8;
 constexpr int MNW_MAX_CHUNKS = 16;
+constexpr int MNW_UNROLL = 4;                     // chunks whose loads are in flight together
 
 // v <- RN(v / S) for 8 values of one block with (S, RN(1/S)), as nv_divide
 __device__ __forceinline__ void divide8(float* v, float2 SY) {
@@ -241,8 +244,13 @@ __device__ __forceinline__ void divide8(float* v, float2 SY) {
     }
 }
 
+__device__ __forceinline__ void unpack8(const uint4& w, float* v) {
+    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+}
+
 template <int FMT, bool SR, int PASS>
-__global__ void __launch_bounds__(MNW_WARPS * 32, 2)
+__global__ void __launch_bounds__(MNW_WARPS * 32, SR ? 3 : 4)   // the Philox words need more registers
 mxnorm_warp_kernel(const MxNormArgs a) {
     constexpr int BLK = (FMT == MXFP4) ? 32 : 16;
     constexpr int LPB = BLK / 8;                       // lanes per block
@@ -260,24 +268,23 @@ mxnorm_warp_kernel(const MxNormArgs a) {
     const int64_t warps = (int64_t)gridDim.x * MNW_WARPS;
     for (int64_t row = (int64_t)blockIdx.x * MNW_WARPS + (threadIdx.x >> 5); row < a.rows; row += warps) {
         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.x) + row * a.ld) + lane;
-        uint4 w[MNW_MAX_CHUNKS];
-#pragma unroll
-        for (int i = 0; i < MNW_MAX_CHUNKS; ++i)
-            if (i < nch) w[i] = __ldg(src + 32 * i);
 
         float rho;
         if (PASS == 2) {
             rho = a.rho[row];
         } else {
-            double part[MNW_MAX_CHUNKS];
+            double mine = 0.0;                        // lane i: the sum of chunk i
             float rmax = 0.0f;
+            for (int i0 = 0; i0 < nch; i0 += MNW_UNROLL) {
+                uint4 w[MNW_UNROLL];
 #pragma unroll
-            for (int i = 0; i < MNW_MAX_CHUNKS; ++i) {
-                part[i] = 0.0;
-                if (i < nch) {
+                for (int u = 0; u < MNW_UNROLL; ++u)
+                    if (i0 + u < nch) w[u] = __ldg(src + 32 * (i0 + u));
+#pragma unroll
+                for (int u = 0; u < MNW_UNROLL; ++u) {
+                    if (i0 + u >= nch) break;
                     float v[8];
-                    v[0] = bf16_lo(w[i].x); v[1] = bf16_hi(w[i].x); v[2] = bf16_lo(w[i].y); v[3] = bf16_hi(w[i].y);
-                    v[4] = bf16_lo(w[i].z); v[5] = bf16_hi(w[i].z); v[6] = bf16_lo(w[i].w); v[7] = bf16_hi(w[i].w);
+                    unpack8(w[u], v);
                     float m = absmax_n<8>(v);
 #pragma unroll
                     for (int sh = 1; sh < LPB; sh <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, sh));
@@ -286,15 +293,13 @@ mxnorm_warp_kernel(const MxNormArgs a) {
                     // the chunk's subtree: butterfly over its blocks, in block order
 #pragma unroll
                     for (int sh = LPB; sh < 32; sh <<= 1) t = __dadd_rn(t, __shfl_xor_sync(0xffffffffu, t, sh));
-                    part[i] = t;
+                    if (lane == i0 + u) mine = t;
                 }
             }
-            // the chunk sums, pairwise over a power-of-two count (zeros past nch)
+            // the chunk sums, pairwise over 16 lanes (zeros past the last chunk)
 #pragma unroll
-            for (int wdt = 1; wdt < MNW_MAX_CHUNKS; wdt <<= 1)
-#pragma unroll
-                for (int i = 0; i + wdt < MNW_MAX_CHUNKS; i += 2 * wdt) part[i] = __dadd_rn(part[i], part[i + wdt]);
-            const double S = part[0];
+            for (int sh = 1; sh < MNW_MAX_CHUNKS; sh <<= 1) mine = __dadd_rn(mine, __shfl_xor_sync(0xffffffffu, mine, sh));
+            const double S = __shfl_sync(0xffffffffu, mine, 0);
             rho = 1.0f;
             if (S > 0.0) {
                 const double mean = __ddiv_rn(S, (double)a.K);
@@ -314,49 +319,55 @@ mxnorm_warp_kernel(const MxNormArgs a) {
 
         // ---- the cast of y = RN(x * rho)
         const float2 rr = make_float2(rho, rho);
+        for (int i0 = 0; i0 < nch; i0 += MNW_UNROLL) {
+            uint4 w[MNW_UNROLL];
 #pragma unroll
-        for (int i = 0; i < MNW_MAX_CHUNKS; ++i) {
-            if (i >= nch) break;
-            float v[8];
-            v[0] = bf16_lo(w[i].x); v[1] = bf16_hi(w[i].x); v[2] = bf16_lo(w[i].y); v[3] = bf16_hi(w[i].y);
-            v[4] = bf16_lo(w[i].z); v[5] = bf16_hi(w[i].z); v[6] = bf16_lo(w[i].w); v[7] = bf16_hi(w[i].w);
-            float mx = absmax_n<8>(v);
+            for (int u = 0; u < MNW_UNROLL; ++u)
+                if (i0 + u < nch) w[u] = __ldg(src + 32 * (i0 + u));
 #pragma unroll
-            for (int sh = 1; sh < LPB; sh <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
+            for (int u = 0; u < MNW_UNROLL; ++u) {
+                const int i = i0 + u;
+                if (i >= nch) break;
+                float v[8];
+                unpack8(w[u], v);
+                float mx = absmax_n<8>(v);
 #pragma unroll
-            for (int j = 0; j < 8; j += 2) {
-                const float2 y = mul2(make_float2(v[j], v[j + 1]), rr);
-                v[j] = y.x;
-                v[j + 1] = y.y;
-            }
-            const float my = __fmul_rn(mx, rho);          // the block's max |y|
-            uint32_t sb;
-            if (FMT == MXFP4) {
-                int e = (my > 0.0f) ? ilogbf(my) - 2 : -127;
-                e = max(-127, min(127, e));
-                sb = (uint32_t)(e + 127);
-                const float inv = (e <= 126) ? __uint_as_float((uint32_t)(127 - e) << 23) : __uint_as_float(0x00400000u);
+                for (int sh = 1; sh < LPB; sh <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
 #pragma unroll
                 for (int j = 0; j < 8; j += 2) {
-                    const float2 t = mul2(make_float2(v[j], v[j + 1]), make_float2(inv, inv));
-                    v[j] = t.x;
-                    v[j + 1] = t.y;
+                    const float2 y = mul2(make_float2(v[j], v[j + 1]), rr);
+                    v[j] = y.x;
+                    v[j + 1] = y.y;
                 }
-            } else {
-                block_scale_codes<FMT, 1>(&my, ref_t, &sb);
-                divide8(v, table.e[sb]);
+                const float my = __fmul_rn(mx, rho);          // the block's max |y|
+                uint32_t sb;
+                if (FMT == MXFP4) {
+                    int e = (my > 0.0f) ? ilogbf(my) - 2 : -127;
+                    e = max(-127, min(127, e));
+                    sb = (uint32_t)(e + 127);
+                    const float inv = (e <= 126) ? __uint_as_float((uint32_t)(127 - e) << 23) : __uint_as_float(0x00400000u);
+#pragma unroll
+                    for (int j = 0; j < 8; j += 2) {
+                        const float2 t = mul2(make_float2(v[j], v[j + 1]), make_float2(inv, inv));
+                        v[j] = t.x;
+                        v[j + 1] = t.y;
+                    }
+                } else {
+                    block_scale_codes<FMT, 1>(&my, ref_t, &sb);
+                    divide8(v, table.e[sb]);
+                }
+                uint32_t rnd[8];
+                if (SR) {
+                    const uint64_t e0 = (uint64_t)row * (uint64_t)C + (uint64_t)(256 * i + 8 * lane);   // a multiple of 8
+                    const uint4 w0 = sr_words(e0 >> 2, a.tensor_id, a.keys);
+                    const uint4 w1 = sr_words((e0 >> 2) + 1, a.tensor_id, a.keys);
+                    rnd[0] = w0.x; rnd[1] = w0.y; rnd[2] = w0.z; rnd[3] = w0.w;
+                    rnd[4] = w1.x; rnd[5] = w1.y; rnd[6] = w1.z; rnd[7] = w1.w;
+                }
+                const uint32_t word = encode8<FMT, SR>(v, rnd);
+                *reinterpret_cast<uint32_t*>(a.codes + row * (C / 2) + 128 * i + 4 * lane) = word;
+                if ((lane & (LPB - 1)) == 0) a.scales[sf_offset(row, (256 / BLK) * i + lane / LPB, a.nb4)] = (uint8_t)sb;
             }
-            uint32_t rnd[8];
-            if (SR) {
-                const uint64_t e0 = (uint64_t)row * (uint64_t)C + (uint64_t)(256 * i + 8 * lane);   // a multiple of 8
-                const uint4 w0 = sr_words(e0 >> 2, a.tensor_id, a.keys);
-                const uint4 w1 = sr_words((e0 >> 2) + 1, a.tensor_id, a.keys);
-                rnd[0] = w0.x; rnd[1] = w0.y; rnd[2] = w0.z; rnd[3] = w0.w;
-                rnd[4] = w1.x; rnd[5] = w1.y; rnd[6] = w1.z; rnd[7] = w1.w;
-            }
-            const uint32_t word = encode8<FMT, SR>(v, rnd);
-            *reinterpret_cast<uint32_t*>(a.codes + row * (C / 2) + 128 * i + 4 * lane) = word;
-            if ((lane & (LPB - 1)) == 0) a.scales[sf_offset(row, (256 / BLK) * i + lane / LPB, a.nb4)] = (uint8_t)sb;
         }
     }
 }
@@ -369,7 +380,7 @@ bool mxnorm_warp_fits(bool bf16, int64_t cols, int64_t ld) {
 template <int FMT, bool SR, int PASS>
 cudaError_t launch_mn_warp(const MxNormArgs& a, cudaStream_t s) {
     int64_t grid = (a.rows + MNW_WARPS - 1) / MNW_WARPS;
-    const int64_t cap = (int64_t)num_sms() * 2;
+    const int64_t cap = (int64_t)num_sms() * (SR ? 3 : 4);
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     mxnorm_warp_kernel<FMT, SR, PASS><<<(unsigned)grid, MNW_WARPS * 32, 0, s>>>(a);
