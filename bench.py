@@ -339,6 +339,32 @@ def fprop_component(fp4, device, flush, peaks, reps):
         "rotate_kernel_alone_ms": rot_only,
         "fused_over_none": fused / none, "unfused_over_none": unf / none,
         "pages": "fused ~1.06-1.07x, unfused ~1.4-1.6x of standalone quantization (SM90/SM100; sizes not stated)"}
+    # the two passes of the NVFP4 + H16 quantization of X on their own, each
+    # against its own bytes: the rotated amax (fp4_amax, one read) and the
+    # quantization given that amax (one read, codes and scales written), beside
+    # the one-launch call's two reads
+    amax = torch.zeros(1, dtype=torch.float32, device=device)
+    H16 = fp4.FP4_ROT_H16
+
+    def amax_only():
+        amax.zero_()
+        fp4.fp4_amax(w.X, fp4.FP4_IN_BF16, M, K, K, H16, 1, 0, amax)
+
+    t_amax = _median_ms(amax_only, flush, reps)
+    t_given = _median_ms(lambda: fp4.quantize(w.X, NV, RT, H16, axis=1, tensor_amax=amax, out=qx), flush, reps)
+    t_fused = _median_ms(lambda: fp4.quantize(w.X, NV, RT, H16, axis=1, out=qx, workspace=ws), flush, reps)
+    read_b = M * K * 2.0
+    one = qbytes(M * K, 2, NV)
+    two = qbytes(M * K, 2, NV, reads=2)
+    hbm = peaks["hbm"]
+    out["quantize_passes"] = {
+        "tensor": "X bf16 %dx%d, NVFP4 + H16, RTNE" % (M, K),
+        "amax_only": {"ms": t_amax, "gbs": read_b / (t_amax * 1e6), "frac_hbm": read_b / (t_amax * 1e6) / hbm,
+                      "bytes": "1 read (the memset of the amax word included in the time)"},
+        "quantize_given_amax": {"ms": t_given, "gbs": one / (t_given * 1e6), "frac_hbm": one / (t_given * 1e6) / hbm,
+                                "bytes": "1 read, codes and scales written"},
+        "one_launch": {"ms": t_fused, "gbs": two / (t_fused * 1e6), "frac_hbm": two / (t_fused * 1e6) / hbm,
+                       "bytes": "2 reads (the second mostly from L2), codes and scales written"}}
     del w, Xr
     torch.cuda.empty_cache()
     return out

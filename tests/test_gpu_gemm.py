@@ -104,11 +104,12 @@ def test_pair_and_single_cta_tiles_give_the_same_bits(fp4, fmt, shape):
     assert torch.equal(out[True].view(torch.int32), out[False].view(torch.int32))
 
 
-def test_gemm_ldc_larger_than_n(fp4):
-    a, b = rand(128, 512, 1), rand(256, 512, 2)
+@pytest.mark.parametrize("M", [128, 256])              # 256: CTA-pair tiles, C written by tiled stores
+def test_gemm_ldc_larger_than_n(fp4, M):
+    a, b = rand(M, 512, 1), rand(256, 512, 2)
     qa, qb = oracle_quantize(a, fmt=NV), oracle_quantize(b, fmt=NV)
     C64, bound = oracle.gemm(qa, qb)
-    out = torch.full((128, 264), 7.0, dtype=torch.float32, device="cuda")
+    out = torch.full((M, 264), 7.0, dtype=torch.float32, device="cuda")
     fp4.gemm(upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb), fp4.FP4_OUT_F32,
              out=out[:, :256])
     torch.cuda.synchronize()

@@ -75,8 +75,9 @@ def test_requantize_writes_only_its_outputs(fp4):
 
 @pytest.mark.parametrize("K", [512, 384])              # 384: the last K stage is half a stage
 @pytest.mark.parametrize("fmt,db", [(0, False), (1, False), (1, True)])
-def test_gemm_writes_only_c_rows_and_columns(fp4, fmt, db, K):
-    M, N, ldc = 256, 384, 392                            # ldc > N: 8 padding columns per row
+@pytest.mark.parametrize("N,ldc", [(384, 392), (512, 520)])   # 512: CTA-pair tiles (not for the double block)
+def test_gemm_writes_only_c_rows_and_columns(fp4, fmt, db, K, N, ldc):
+    M = 256                                              # ldc > N: 8 padding columns per row
     g = torch.Generator().manual_seed(fmt)
     a = torch.randn((M, K), generator=g).to(torch.bfloat16).cuda()
     b = torch.randn((N, K), generator=g).to(torch.bfloat16).cuda()
