@@ -62,22 +62,26 @@ __global__ void build_mask_kernel(const int32_t* __restrict__ ch, int64_t n, int
     }
 }
 
-// FP8 pass 1: amax of the gathered channels
+// FP8 pass 1: amax of the gathered channels.  Rows are spread over the CTAs
+// (grid-stride) and a row's channels over the threads, so a thread reads the
+// channel list once per row from L1 and forms one 64-bit row offset per row.
 __global__ void __launch_bounds__(OC_THREADS)
 fp8_amax_kernel(const void* __restrict__ x, bool bf16, int64_t rows, int64_t cols, int64_t ld,
                 const int32_t* __restrict__ ch, int64_t n, unsigned int* __restrict__ amax) {
     float m = 0.0f;
-    const int64_t total = rows * n;
-    for (int64_t i = (int64_t)blockIdx.x * OC_THREADS + threadIdx.x; i < total; i += (int64_t)gridDim.x * OC_THREADS) {
-        const int64_t r = i / n, j = i - r * n;
-        const int32_t c = __ldg(ch + j);
-        if (c >= 0 && c < cols) m = fmaxf(m, fabsf(load_as_f32(x, bf16, r * ld + c)));
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int64_t base = r * ld;
+        for (int64_t j = threadIdx.x; j < n; j += OC_THREADS) {
+            const int32_t c = __ldg(ch + j);
+            if (c >= 0 && c < cols) m = fmaxf(m, fabsf(load_as_f32(x, bf16, base + c)));
+        }
     }
     const uint32_t b = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
     if ((threadIdx.x & 31) == 0 && b) atomicMax(amax, b);
 }
 
-// FP8 pass 2: the codes of [rows, k8] (zero past n) and the tensor scale
+// FP8 pass 2: the codes of [rows, k8] (zero past n) and the tensor scale; two
+// codes per thread step (one e4m3x2 conversion), k8 even
 __global__ void __launch_bounds__(OC_THREADS)
 fp8_quantize_kernel(const void* __restrict__ x, bool bf16, int64_t rows, int64_t cols, int64_t ld,
                     const int32_t* __restrict__ ch, int64_t n, int64_t k8, const float* __restrict__ amax,
@@ -85,22 +89,22 @@ fp8_quantize_kernel(const void* __restrict__ x, bool bf16, int64_t rows, int64_t
     float s8 = __fdiv_rn(*amax, 448.0f);
     if (!(s8 > 0.0f)) s8 = 1.0f;
     if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s8;
-    // two codes per thread step (one e4m3x2 conversion), k8 even
-    const int64_t pairs = k8 / 2, total = rows * pairs;
-    for (int64_t i = (int64_t)blockIdx.x * OC_THREADS + threadIdx.x; i < total; i += (int64_t)gridDim.x * OC_THREADS) {
-        const int64_t r = i / pairs, j = (i - r * pairs) * 2;
-        float v[2];
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int64_t base = r * ld;
+        for (int64_t j = 2 * threadIdx.x; j < k8; j += 2 * OC_THREADS) {
+            float v[2];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            v[e] = 0.0f;
-            if (j + e < n) {
-                const int32_t c = __ldg(ch + j + e);
-                if (c >= 0 && c < cols) v[e] = __fdiv_rn(load_as_f32(x, bf16, r * ld + c), s8);
+            for (int e = 0; e < 2; ++e) {
+                v[e] = 0.0f;
+                if (j + e < n) {
+                    const int32_t c = __ldg(ch + j + e);
+                    if (c >= 0 && c < cols) v[e] = __fdiv_rn(load_as_f32(x, bf16, base + c), s8);
+                }
             }
+            uint16_t pk;
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pk) : "f"(v[1]), "f"(v[0]));
+            *reinterpret_cast<uint16_t*>(codes + r * k8 + j) = pk;
         }
-        uint16_t pk;
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pk) : "f"(v[1]), "f"(v[0]));
-        *reinterpret_cast<uint16_t*>(codes + r * k8 + j) = pk;
     }
 }
 
@@ -131,12 +135,15 @@ cudaError_t launch_channel_mask(const int32_t* ch, int64_t n, int64_t cols, uint
 cudaError_t launch_fp8_gather(const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld, const int32_t* ch,
                               int64_t n, int64_t k8, unsigned int* amax_word, uint8_t* codes, float* scale,
                               cudaStream_t s) {
+    // one CTA per row at a time, at most 8 CTAs per SM
+    const int64_t cap = (int64_t)num_sms() * 8;
+    const unsigned grid = (unsigned)(rows < cap ? (rows > 0 ? rows : 1) : cap);
     if (n > 0) {
-        fp8_amax_kernel<<<grid_for(rows * n, 8), OC_THREADS, 0, s>>>(x, bf16, rows, cols, ld, ch, n, amax_word);
+        fp8_amax_kernel<<<grid, OC_THREADS, 0, s>>>(x, bf16, rows, cols, ld, ch, n, amax_word);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    fp8_quantize_kernel<<<grid_for(rows * (k8 / 2), 8), OC_THREADS, 0, s>>>(
+    fp8_quantize_kernel<<<grid, OC_THREADS, 0, s>>>(
         x, bf16, rows, cols, ld, ch, n, k8, reinterpret_cast<const float*>(amax_word), codes, scale);
     return cudaGetLastError();
 }
