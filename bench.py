@@ -151,7 +151,7 @@ class LayerStep:
     """Device buffers and the step of the layer workload: per linear, the six
     NVFP4 + H16 operands and the Fprop, Dgrad and Wgrad GEMMs."""
 
-    def __init__(self, fp4, device, seed=0, fmt=None, host=None):
+    def __init__(self, fp4, device, seed=0, fmt=None, host=None, both_axes=True):
         self.fp4 = fp4
         self.fmt = fp4.FP4_NVFP4 if fmt is None else fmt
         self.device = device
@@ -171,14 +171,34 @@ class LayerStep:
                 calls.append(dict(x=tn, axis=axis, rounding=fp4.FP4_SR if sr else fp4.FP4_RTNE,
                                   tensor_id=workloads.layer_tensor_id(index, role), name="%s_ax%d" % (tn, axis)))
                 self.quant_bytes += qbytes(R * C, 2, self.fmt, reads=2)
-                self.launches += quantize_kernels(axis, True)
             outs = []
             for gname, ra, rb, bf16 in GEMMS:
                 M, N, K = qs[ra]["lines"], qs[rb]["lines"], qs[ra]["K"]
                 outs.append(torch.empty((M, N), dtype=torch.bfloat16 if bf16 else torch.float32, device=device))
                 self.flop += 2.0 * M * N * K
-                self.launches += 1
-            self.linears.append(dict(name=name, t=t, qs=qs, calls=calls, outs=outs))
+            # both-axes calls: each tensor once, its row operand and its column operand together
+            both = []
+            for tn in dict.fromkeys(c["x"] for c in calls):
+                rrole = next(r for r, c in enumerate(calls) if c["x"] == tn and c["axis"] == 1)
+                crole = next(r for r, c in enumerate(calls) if c["x"] == tn and c["axis"] == 0)
+                both.append(dict(x=tn, rows=rrole, cols=crole, name="%s_both" % tn))
+            self.linears.append(dict(name=name, t=t, qs=qs, calls=calls, both=both, outs=outs))
+        self.set_both_axes(both_axes)
+
+    def set_both_axes(self, on):
+        """Quantize each tensor along both axes in one call (fp4_quantize_both_axes,
+        3 calls per linear) or each operand on its own (fp4_quantize, 6 calls)."""
+        self.both_axes = bool(on)
+        n_lin = len(self.linears)
+        self.launches = n_lin * (3 if self.both_axes else len(OPERANDS)) + n_lin * len(GEMMS)
+
+    def quantize_both(self, lin, k):
+        b = lin["both"][k]
+        cr, cc = lin["calls"][b["rows"]], lin["calls"][b["cols"]]
+        self.fp4.quantize_both_axes(lin["t"][b["x"]], self.fmt, self.fp4.FP4_ROT_H16, seed=0,
+                                    rounding_rows=cr["rounding"], tensor_id_rows=cr["tensor_id"],
+                                    rounding_cols=cc["rounding"], tensor_id_cols=cc["tensor_id"],
+                                    out_rows=lin["qs"][b["rows"]], out_cols=lin["qs"][b["cols"]], workspace=self.ws)
 
     def quantize(self, lin, role):
         c = lin["calls"][role]
@@ -194,9 +214,13 @@ class LayerStep:
         """The step's calls in order: (kind, linear name, call name, fn)."""
         out = []
         for lin in self.linears:
-            for role in range(len(OPERANDS)):
-                kind = "quant_rows" if lin["calls"][role]["axis"] == 1 else "quant_cols"
-                out.append((kind, lin["name"], lin["calls"][role]["name"], role, lin))
+            if self.both_axes:
+                for k, b in enumerate(lin["both"]):
+                    out.append(("quant_both", lin["name"], b["name"], k, lin))
+            else:
+                for role in range(len(OPERANDS)):
+                    kind = "quant_rows" if lin["calls"][role]["axis"] == 1 else "quant_cols"
+                    out.append((kind, lin["name"], lin["calls"][role]["name"], role, lin))
             for g in range(len(GEMMS)):
                 out.append(("gemm", lin["name"], GEMMS[g][0], g, lin))
         return out
@@ -205,13 +229,19 @@ class LayerStep:
         kind, _, _, i, lin = c
         if kind == "gemm":
             self.gemm(lin, i)
+        elif kind == "quant_both":
+            self.quantize_both(lin, i)
         else:
             self.quantize(lin, i)
 
     def step(self):
         for lin in self.linears:
-            for role in range(len(OPERANDS)):
-                self.quantize(lin, role)
+            if self.both_axes:
+                for k in range(len(lin["both"])):
+                    self.quantize_both(lin, k)
+            else:
+                for role in range(len(OPERANDS)):
+                    self.quantize(lin, role)
             for g in range(len(GEMMS)):
                 self.gemm(lin, g)
 
@@ -259,6 +289,15 @@ def per_call_split(layer, flush, reps, peaks):
             work = 2.0 * M * N * K
             e = {"ms": t, "tflops": work / (t * 1e-3) / 1e12, "frac_fp4": work / (t * 1e-3) / 1e12 / fp4_peak,
                  "shape": [M, N, K], "launches": 1}
+        elif kind == "quant_both":
+            b = lin["both"][i]
+            x = lin["t"][b["x"]]
+            # the input read twice (amax pass, quantize pass) for both axes; both outputs written
+            work = 2 * x.numel() * 2 + 2 * (qbytes(x.numel(), 2, layer.fmt, reads=0))
+            e = {"ms": t, "gbs": work / (t * 1e6), "frac_hbm": work / (t * 1e6) / peaks["hbm"],
+                 "bytes": "2 reads (amax pass + quantize, both axes at once) + both outputs", "launches": 1,
+                 "rounding": "rows %s, columns %s" % tuple("SR" if lin["calls"][b[a]]["rounding"] else "RTNE"
+                                                            for a in ("rows", "cols"))}
         else:
             x = lin["t"][lin["calls"][i]["x"]]
             work = qbytes(x.numel(), 2, layer.fmt, reads=2)
@@ -412,6 +451,21 @@ def run_gpu(args, rank, world, device, host):
 
     table, fam = per_call_split(layer, flush, max(3, min(args.steps, 10)), peaks)
 
+    # the same step with each of the 24 operands quantized by its own call
+    # (fp4_quantize along one axis; each bf16 tensor is then read for each axis)
+    layer.set_both_axes(False)
+    sep_reps = max(3, min(args.steps, 10))
+    layer.step()
+    torch.cuda.synchronize()
+    sep_ms = statistics.median(time_steps(layer.step, flush, sep_reps))
+    _, sep_fam = per_call_split(layer, flush, sep_reps, peaks)
+    layer.set_both_axes(True)
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    separate = {"ms_per_step": round(sep_ms, 4), "value": round(layer.flop / (sep_ms * 1e-3) / 1e12, 2),
+                "families_ms": {k: round(v["ms"], 4) for k, v in sep_fam.items()},
+                "how": "24 fp4_quantize calls (one axis each, with its tensor amax) + the 12 GEMMs, median of %d "
+                       "event-timed steps, L2 flushed before each" % sep_reps}
+
     # end to end through the public API: every step copies its inputs (X, W and
     # dY of the four linears) from pinned host memory and its results (the 12
     # GEMM outputs) back.  Two sets of device buffers on three streams
@@ -419,7 +473,8 @@ def run_gpu(args, rank, world, device, host):
     # i-1's results cross PCIe while step i computes.
     e2e_steps = 0 if args.no_e2e else 4
     if e2e_steps == 0:
-        return finish_line(args, rank, world, device, layer, fam, table, total_ms, None, 0, 0, clocks, status, peaks)
+        return finish_line(args, rank, world, device, layer, fam, table, total_ms, None, 0, 0, clocks, status, peaks,
+                           separate)
     hin = [{k: v.pin_memory() for k, v in h.items()} for h in host]
     hout = [[[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in lin["outs"]] for lin in layer.linears]
             for _ in range(2)]
@@ -467,10 +522,12 @@ def run_gpu(args, rank, world, device, host):
     del slots, second, hout
     torch.cuda.empty_cache()
 
-    return finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, h2d, d2h, clocks, status, peaks)
+    return finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, h2d, d2h, clocks, status, peaks,
+                       separate)
 
 
-def finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, h2d, d2h, clocks, status, peaks):
+def finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, h2d, d2h, clocks, status, peaks,
+                separate=None):
     """Max over ranks of the timings, then rank 0's JSON line."""
     from fp4_block_scaled_h16_b200 import fp4
     t = torch.tensor([total_ms, e2e_ms if e2e_ms is not None else 0.0], dtype=torch.float64, device=device)
@@ -495,8 +552,10 @@ def finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, 
                 "achieved_is": "GEMM FLOP of the step / summed mean event time of its 12 GEMM launches",
                 "peak_is": "%s bf16 burst %.1f TFLOP/s x 4 (nominal fp4 / bf16 ratio)" % (peaks["src"], peaks["bf16"])}
     else:
-        roof = {"bound": "hbm", "kernel": ("quant_rows_kernel" if dom == "quant_rows" else
-                                           "quant_cols_kernel (amax + quantize)") + ", 12 calls per step",
+        roof = {"bound": "hbm", "kernel": {"quant_rows": "quant_rows_kernel, 12 calls per step",
+                                           "quant_cols": "quant_cols_kernel (amax + quantize), 12 calls per step",
+                                           "quant_both": "quant_cols_kernel, both axes (amax + quantize of the rows "
+                                                         "and the columns), 12 calls per step"}[dom],
                 "achieved": round(f["gbs"], 1), "peak": round(peaks["hbm"], 1), "unit": "GB/s",
                 "frac": round(f["gbs"] / peaks["hbm"], 4), "traffic": None,
                 "achieved_is": "algorithmic bytes (input read twice: amax pass + quantize; codes and "
@@ -516,14 +575,14 @@ def finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, 
                    "format": "NVFP4", "rotation": "H16 on all three GEMMs",
                    "rounding": "RTNE; SR on the Wgrad operands", "out": "bf16 (Fprop, Dgrad), f32 (Wgrad)",
                    "gemm_flop_per_step": layer.flop,
-                   "value_is": "GEMM FLOP of the step / whole step time (24 quantize calls, each with its "
-                               "tensor amax, + 12 GEMMs)",
+                   "value_is": "GEMM FLOP of the step / whole step time (the 24 NVFP4 operands from 12 "
+                               "both-axes quantize calls, each axis with its own tensor amax, + 12 GEMMs)",
                    "l2": "flushed before every step (256 MiB write, then 256 MiB read, outside the timed "
                          "events); the step's 1.6 GB of inputs exceed L2",
                    "launch": "the step replayed as one CUDA graph" if args.graph else "eager launches",
                    "parallelism": "independent layer per GPU" if world > 1 else "single GPU"},
         "roofline": roof,
-        "components": {"per_call": table},
+        "components": {"per_call": table, "separate_axes": separate},
         "e2e": ({"value": round(world * layer.flop / (e2e_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                  "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_max, 3),
                  "how": "fp4.quantize / fp4.gemm on the layer's inputs copied from pinned host memory every step, "

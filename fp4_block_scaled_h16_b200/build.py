@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp4.so")
 SOURCES = ["fp4_api.cu", "quantize.cu", "quantize_rows_f32.cu", "quantize_cols_bf16.cu", "quantize_cols_f32.cu",
            "requantize_cols.cu", "gemm.cu", "gemm_db.cu", "quantize_noalloc.cu", "rotate.cu", "mxnorm.cu", "ufp4_split.cu",
-           "outctl.cu", "gemm_outctl.cu", "gemm_pair.cu"]
+           "outctl.cu", "gemm_outctl.cu", "gemm_pair.cu", "quantize_dual.cu"]
 HEADERS = ["fp4_device.cuh", "internal.h", "sm100.cuh", "quant_common.cuh", "quant_rows.cuh", "quant_cols.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

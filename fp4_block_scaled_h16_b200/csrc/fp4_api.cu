@@ -274,6 +274,70 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
     return FP4_OK;
 }
 
+fp4_status_t fp4_quantize_both_axes(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
+                                    fp4_format_t format, fp4_rotation_t rotation, uint64_t seed,
+                                    fp4_rounding_t rounding_rows, uint32_t tensor_id_rows, uint8_t* codes_rows,
+                                    uint8_t* scales_rows, float* tensor_scale_rows, fp4_rounding_t rounding_cols,
+                                    uint32_t tensor_id_cols, uint8_t* codes_cols, uint8_t* scales_cols,
+                                    float* tensor_scale_cols, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+    fp4_status_t st = check_input(x, in_dtype, rows, cols, ld, rotation, 1);
+    if (st != FP4_OK) return st;
+    if (format < FP4_MXFP4 || format > FP4_UFP4) return FP4_ERR_INVALID_ARG;
+    if (rounding_rows != FP4_RTNE && rounding_rows != FP4_SR) return FP4_ERR_INVALID_ARG;
+    if (rounding_cols != FP4_RTNE && rounding_cols != FP4_SR) return FP4_ERR_INVALID_ARG;
+    if (!tensor_scale_rows || !tensor_scale_cols) return FP4_ERR_INVALID_ARG;
+    if (in_dtype != FP4_IN_BF16 || format == FP4_MXFP4) return FP4_ERR_UNSUPPORTED;
+    if (rotation != FP4_ROT_NONE && rotation != FP4_ROT_H16) return FP4_ERR_UNSUPPORTED;
+    if (rows % 16 || cols % 64) return FP4_ERR_UNSUPPORTED_SHAPE;
+    const bool empty = rows == 0 || cols == 0;
+    if (!empty && (!codes_rows || !scales_rows || !codes_cols || !scales_cols)) return FP4_ERR_INVALID_ARG;
+    if ((codes_rows && !aligned16(codes_rows)) || (codes_cols && !aligned16(codes_cols)) ||
+        ((uintptr_t)tensor_scale_rows & 3u) || ((uintptr_t)tensor_scale_cols & 3u))
+        return FP4_ERR_MISALIGNED;
+    if (!empty) {
+        if (!workspace || workspace_bytes < 256) return FP4_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    }
+    int dev;
+    if ((st = device_ready(&dev)) != FP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (empty) {
+        static const float one = 1.0f;
+        if (cudaMemcpyAsync(tensor_scale_rows, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(tensor_scale_cols, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return FP4_ERR_CUDA;
+        return FP4_OK;
+    }
+    // workspace words: 0 the column-axis amax, 1 the grid-barrier count, 2 the row-axis amax
+    if (cudaMemsetAsync(workspace, 0, 3 * sizeof(unsigned int), s) != cudaSuccess) return FP4_ERR_CUDA;
+    unsigned int* words = static_cast<unsigned int*>(workspace);
+    QuantArgs a{};
+    a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
+    a.L = cols; a.K = rows;
+    a.nb4 = ((rows / 16) + 3) / 4;
+    a.codes = codes_cols; a.scales = scales_cols;
+    a.tensor_scale_out = tensor_scale_cols;
+    a.amax_out = words;
+    a.grid_count = words + 1;
+    a.amax_in = reinterpret_cast<const float*>(words);
+    a.keys = make_keys(seed);
+    a.tensor_id = tensor_id_cols;
+    a.sign_mask = sign_mask_of(rotation, seed);
+    a.err = device_error_word();
+    a.wait_limit = g_wait_limit;
+    RowOut ro{};
+    ro.codes = codes_rows; ro.scales = scales_rows;
+    ro.tensor_scale_out = tensor_scale_rows;
+    ro.amax_out = words + 2;
+    ro.nb4 = ((cols / 16) + 3) / 4;
+    ro.tensor_id = tensor_id_rows;
+    if (launch_both_axes(a, ro, format, rounding_cols == FP4_SR, rounding_rows == FP4_SR, rot_size(rotation), s) !=
+        cudaSuccess)
+        return FP4_ERR_CUDA;
+    return FP4_OK;
+}
+
 fp4_status_t fp4_mxnorm_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols, int64_t ld,
                                  fp4_format_t format, fp4_rounding_t rounding, int p, float c, uint64_t seed,
                                  uint32_t tensor_id, uint8_t* codes, uint8_t* scales, float* tensor_scale,

@@ -440,7 +440,7 @@ bool make_c_map(CUtensorMap* m, void* c, bool bf16, int64_t M, int64_t N, int64_
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld) {
+bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld, bool swizzle128) {
     auto fn = encode_fn();
     if (!fn) return false;
     const int64_t es = bf16 ? 2 : 4;
@@ -449,7 +449,8 @@ bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int6
     cuuint32_t box[2] = {64u, 128u};
     cuuint32_t estr[2] = {1u, 1u};
     return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(x),
-              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              (swizzle128 && bf16) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -55,9 +55,24 @@ template <bool BF16>
 cudaError_t launch_cols_amax(const QuantArgs& a, int rot_n, bool signs, cudaStream_t s);
 template <bool BF16>
 cudaError_t launch_cols_fused(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, cudaStream_t s);
+// both axes of a bf16 tensor in one cooperative launch (quantize_dual.cu): the
+// QuantArgs describe the column-axis result, RowOut the row-axis result
+// (rows of `cols` elements)
+struct RowOut {
+    uint8_t* codes;             // [rows, cols / 2]
+    uint8_t* scales;            // tiled layout, nb4 groups of 4 blocks per row
+    float* tensor_scale_out;
+    unsigned int* amax_out;     // the row-rotated amax (atomicMax target, zeroed by the host)
+    int64_t nb4;
+    uint32_t tensor_id;         // SR stream of the row quantization
+};
+cudaError_t launch_both_axes(const QuantArgs& a, const RowOut& ro, int fmt, bool sr_cols, bool sr_rows, int rot_n,
+                             cudaStream_t s);
 // 2-D TMA map over a [rows, cols] input of row pitch ld, box 64 columns x 128
-// rows, no swizzle, zeros past the edges
-bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld);
+// rows, zeros past the edges; swizzle128 (bf16 only): the tile lands with the
+// 128-byte swizzle, 16-byte chunk c of tile row r at chunk c ^ (r % 8)
+bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld,
+                    bool swizzle128 = false);
 // the same two along axis 0 of the dequantized source (a.src_*)
 cudaError_t launch_requantize_cols(const QuantArgs& a, int fmt, bool sr, int rot_n, bool signs, bool db,
                                    cudaStream_t s);

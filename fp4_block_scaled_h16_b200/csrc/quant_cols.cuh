@@ -22,7 +22,15 @@
 //
 // Modes, as the row axis: quantize with a known tensor amax, the amax alone,
 // or both in one cooperative launch (amax pass, bounded grid barrier, quantize
-// pass over the same tiles in reverse order).  Every wait is bounded by the
+// pass over the same tiles in reverse order).
+//
+// Both axes (DUAL, bf16, fused only): the same launch also quantizes along the
+// rows, from the same tiles, so the tensor crosses HBM once for both layouts.
+// The tiles then land with the 128-byte swizzle (16-byte chunk c of tile row r
+// at chunk c ^ (r % 8)), so that thread t reading tile row t (two 32-element
+// row units, the row quantizer's arithmetic) and the column lanes both read
+// shared memory without bank conflicts.  The row part of each tile runs
+// before the column part copies the tile out and releases its slot.  Every wait is bounded by the
 // wait limit of fp4_set_wait_limit (ring: 16 x, grid barrier: 4 x); whatever
 // way a CTA leaves, thread 0 first waits for every tile load it issued.
 #pragma once
@@ -47,14 +55,16 @@ __device__ __forceinline__ uint32_t qc_grid_limit(uint32_t w) { return w >= (1u 
 // Four CTAs per SM (128 registers).  (Measured on B200: a fifth CTA for the
 // stochastic-rounding variants, at 96 registers with two stages, was no
 // faster: they are bound by their instruction count, not by occupancy.)
-template <bool BF16, bool SR>
+template <bool BF16, bool SR, bool SWZ = false>
 struct ColRing {
     static constexpr int ES = BF16 ? 2 : 4;
     static constexpr int BYTES = QC_ROWS * QC_COLS * ES;        // one tile: 16 KB (bf16) / 32 KB (f32)
     static constexpr int STAGES = BF16 ? 3 : 2;
     static constexpr int CTAS = 4;                              // the launch bound
-    static constexpr int SMEM = STAGES * BYTES + 128 /*alignment*/ + STAGES * 16 /*barriers*/;
+    static constexpr int ALIGN = SWZ ? 1024 : 128;              // the 128-byte swizzle wants 1024-byte stages
+    static constexpr int SMEM = STAGES * BYTES + ALIGN /*alignment*/ + STAGES * 16 /*barriers*/;
 };
+
 
 struct ColTiles {
     int n_tr, n_tc, total;      // row tiles, column tiles, n_tr * n_tc (< 2^31)
@@ -81,22 +91,28 @@ __device__ __forceinline__ float col_of(const float2& p, int c) { return (c & 1)
 
 // ALIGN4 (stochastic rounding only): cols % 4 == 0, so the four columns of a
 // row are one Philox counter; otherwise they may straddle two
-template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE, bool ALIGN4 = true>
-__global__ void __launch_bounds__(QC_THREADS, (ColRing<BF16, SR>::CTAS))
-quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, const ColTiles ct) {
+// DUAL / SR1: also quantize along the rows (rounding SR1), see the file comment
+template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE, bool ALIGN4 = true, bool DUAL = false,
+          bool SR1 = false>
+__global__ void __launch_bounds__(QC_THREADS, (ColRing<BF16, SR, DUAL>::CTAS))
+quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, const ColTiles ct, const RowOut ro) {
     constexpr bool AMAX_ONLY = MODE == QC_AMAX, FUSED = MODE == QC_FUSED;
     static_assert(!FUSED || (FMT != MXFP4 && !DB), "only a tensor-scaled format has an amax pass");
     static_assert(!DB || (FMT == NVFP4 && MODE == QC_QUANT), "double block: NVFP4 quantize only");
-    using Ring = ColRing<BF16, SR>;
+    static_assert(!DUAL || (BF16 && FUSED && ALIGN4), "both axes: bf16, fused launch, cols % 64 == 0");
+    using Ring = ColRing<BF16, SR, DUAL>;
     constexpr int STAGES = Ring::STAGES, BYTES = Ring::BYTES;
     constexpr int BLK = (FMT == MXFP4) ? 32 : 16;
     extern __shared__ uint8_t qc_smem_raw[];
-    uint8_t* buf = qc_smem_raw + ((128u - (sm100::smem_u32(qc_smem_raw) & 127u)) & 127u);
+    constexpr uint32_t AL = (uint32_t)Ring::ALIGN;
+    uint8_t* buf = qc_smem_raw + ((AL - (sm100::smem_u32(qc_smem_raw) & (AL - 1u))) & (AL - 1u));
     uint64_t* full = reinterpret_cast<uint64_t*>(buf + STAGES * BYTES);   // tile landed
     uint64_t* empty = full + STAGES;                                     // every warp has copied it out
     __shared__ ScaleTable table;                        // (S, 1/S) per E4M3 code under s_t
     __shared__ float chunk_max[2][4][QC_COLS];          // double block: 32-row column maxima per warp
     __shared__ float warp_max[QC_THREADS / 32];
+    __shared__ ScaleTable table1;                       // DUAL: the row quantization's table
+    __shared__ float warp_max1[QC_THREADS / 32];
     __shared__ uint32_t grid_verdict;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = lane & 15, h = lane >> 4;
@@ -135,20 +151,29 @@ quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, co
         for (int p = 0; p < STAGES - 1; ++p)
             if (p < nv) issue(tile_of(p), p);
 
-    float tmax = 0.0f;
+    float tmax = 0.0f, tmax1 = 0.0f;
+    ScaleRef ref_t1 = make_ref(1.0f);
     bool ok = true;
     for (int it = 0; it < nv; ++it) {
         if (FUSED && it == n) {
             // end of the amax pass: the CTA's maximum, the grid's, then the
             // tensor scale and its table (every thread of the CTA gets here)
             const uint32_t wbits = __reduce_max_sync(0xffffffffu, __float_as_uint(tmax));
-            if (lane == 0) warp_max[warp] = __uint_as_float(wbits);
+            const uint32_t wbits1 = DUAL ? __reduce_max_sync(0xffffffffu, __float_as_uint(tmax1)) : 0u;
+            if (lane == 0) {
+                warp_max[warp] = __uint_as_float(wbits);
+                if (DUAL) warp_max1[warp] = __uint_as_float(wbits1);
+            }
             const bool failed = __syncthreads_or(!ok);
             if (tid == 0) {
-                float m = 0.0f;
+                float m = 0.0f, m1 = 0.0f;
 #pragma unroll
-                for (int w = 0; w < QC_THREADS / 32; ++w) m = fmaxf(m, warp_max[w]);
+                for (int w = 0; w < QC_THREADS / 32; ++w) {
+                    m = fmaxf(m, warp_max[w]);
+                    if (DUAL) m1 = fmaxf(m1, warp_max1[w]);
+                }
                 if (__float_as_uint(m)) atomicMax(a.amax_out, __float_as_uint(m));
+                if (DUAL && __float_as_uint(m1)) atomicMax(ro.amax_out, __float_as_uint(m1));
                 __threadfence();
                 atomicAdd(a.grid_count, 1u);
                 bool done = false;
@@ -159,6 +184,7 @@ quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, co
                 }
                 if (!done) atomicExch(a.err, 7u);       // FP4_ERR_TIMEOUT
                 warp_max[0] = __uint_as_float(sm100::ld_acquire_gpu(a.amax_out));
+                if (DUAL) warp_max1[0] = __uint_as_float(sm100::ld_acquire_gpu(ro.amax_out));
                 grid_verdict = (done && !failed) ? 1u : 0u;
             }
             __syncthreads();
@@ -169,6 +195,11 @@ quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, co
             ref_t = make_ref(tensor_scale_of(warp_max[0], FMT));
             if (blockIdx.x == 0 && tid == 0 && a.tensor_scale_out) *a.tensor_scale_out = ref_t.s;
             table.build(ref_t.s, tid, QC_THREADS);
+            if (DUAL) {
+                ref_t1 = make_ref(tensor_scale_of(warp_max1[0], FMT));
+                if (blockIdx.x == 0 && tid == 0 && ro.tensor_scale_out) *ro.tensor_scale_out = ref_t1.s;
+                table1.build(ref_t1.s, tid, QC_THREADS);
+            }
             __syncthreads();
         }
         const int t = tile_of(it);
@@ -184,6 +215,54 @@ quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, co
                 break;
             }
         }
+        if (DUAL && got) {
+            // ---- the row axis: thread t quantizes tile row t, two 32-element units
+            const uint8_t* tile = buf + slot * BYTES;
+            const int tr = (int)fast_div((uint32_t)t, ct.tc_m, ct.tc_l), tc = t - tr * ct.n_tc;
+            const int64_t row = (int64_t)tr * QC_ROWS + tid;
+#pragma unroll 1
+            for (int u = 0; u < 2; ++u) {
+                float v1[32];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    // logical chunk 4u + k of row tid sits at chunk (4u + k) ^ (tid % 8)
+                    const uint4 w = *reinterpret_cast<const uint4*>(tile + tid * 128 + (((4 * u + k) ^ (tid & 7)) << 4));
+                    v1[8 * k + 0] = bf16_lo(w.x); v1[8 * k + 1] = bf16_hi(w.x);
+                    v1[8 * k + 2] = bf16_lo(w.y); v1[8 * k + 3] = bf16_hi(w.y);
+                    v1[8 * k + 4] = bf16_lo(w.z); v1[8 * k + 5] = bf16_hi(w.z);
+                    v1[8 * k + 6] = bf16_lo(w.w); v1[8 * k + 7] = bf16_hi(w.w);
+                }
+                if (it < n) {
+                    // rows past the tensor read as zeros and leave the maximum alone
+                    tmax1 = unit_rotated_absmax<32, ROT, SIGNS>(v1, a.sign_mask, tmax1);
+                    continue;
+                }
+                if (row >= R) continue;
+                rotate_unit<32, ROT, SIGNS>(v1, a.sign_mask);
+                float bm[2] = {absmax_n<16>(v1), absmax_n<16>(v1 + 16)};
+                uint32_t sb[2];
+                block_scale_codes<FMT, 2>(bm, ref_t1, sb);
+                const float2 SY[2] = {table1.e[sb[0]], table1.e[sb[1]]};
+                nv_divide<32, ROT>(v1, SY);
+                const int64_t c0 = (int64_t)tc * QC_COLS + 32 * u;      // first column of the unit
+                uint32_t rnd[32];
+                if (SR1) {
+                    const uint64_t i0 = (uint64_t)row * (uint64_t)C + (uint64_t)c0;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint4 w = sr_words((i0 >> 2) + k, ro.tensor_id, a.keys);
+                        rnd[4 * k] = w.x; rnd[4 * k + 1] = w.y; rnd[4 * k + 2] = w.z; rnd[4 * k + 3] = w.w;
+                    }
+                }
+                uint32_t words[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) words[k] = encode8<FMT, SR1>(v1 + 8 * k, rnd + 8 * k);
+                *reinterpret_cast<uint4*>(ro.codes + row * (C / 2) + c0 / 2) = make_uint4(words[0], words[1], words[2], words[3]);
+                // blocks 2j' and 2j'+1 sit side by side in the tiled layout
+                *reinterpret_cast<uint16_t*>(ro.scales + sf_offset(row, c0 / 16, ro.nb4)) = (uint16_t)(sb[0] | (sb[1] << 8));
+            }
+        }
+
         // my 16 rows x 4 columns, out of the slot
         float2 v[16][2];
         if (got) {
@@ -191,7 +270,14 @@ quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, co
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int rr = 32 * warp + 16 * h + j;
-                if (BF16) {
+                if (DUAL) {
+                    // columns 4q .. 4q+3: half (q % 2) of logical chunk q / 2, which
+                    // sits at chunk (q / 2) ^ (rr % 8), and rr % 8 = j % 8
+                    const uint2 w = *reinterpret_cast<const uint2*>(tile + rr * 128 + (((q >> 1) ^ (j & 7)) << 4) +
+                                                                    ((q & 1) << 3));
+                    v[j][0] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
+                    v[j][1] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+                } else if (BF16) {
                     const uint2 w = *reinterpret_cast<const uint2*>(tile + (rr * QC_COLS + 4 * q) * 2);
                     v[j][0] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
                     v[j][1] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
@@ -470,9 +556,6 @@ quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, co
     }
 }
 
-// 2-D TMA map over the [rows, cols] input (row pitch ld elements), box
-// 64 columns x 128 rows, no swizzle, zeros past the edges
-bool make_input_map(CUtensorMap* m, const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld);
 
 template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE, bool ALIGN4>
 cudaError_t launch_cols_k(const QuantArgs& a, cudaStream_t s) {
@@ -508,12 +591,71 @@ cudaError_t launch_cols_k(const QuantArgs& a, cudaStream_t s) {
         if (resident < 1) return cudaErrorInvalidConfiguration;
         QuantArgs ka = a;
         ColTiles kct = ct;
-        void* args[] = {&tm, &ka, &kct};
+        RowOut kro{};
+        void* args[] = {&tm, &ka, &kct, &kro};
         return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3((unsigned)grid),
                                            dim3(QC_THREADS), args, Ring::SMEM, s);
     }
-    kernel<<<(unsigned)grid, QC_THREADS, Ring::SMEM, s>>>(tm, a, ct);
+    kernel<<<(unsigned)grid, QC_THREADS, Ring::SMEM, s>>>(tm, a, ct, RowOut{});
     return cudaGetLastError();
+}
+
+// both axes in one cooperative launch (bf16, NVFP4 / UFP4, cols % 64 == 0):
+// a describes the column-axis result and carries the shared fields, ro the
+// row-axis result; a.amax_out, ro.amax_out and a.grid_count are zeroed words
+template <int FMT, bool SR0, bool SR1, int ROT>
+cudaError_t launch_dual_k(const QuantArgs& a, const RowOut& ro, cudaStream_t s) {
+    using Ring = ColRing<true, SR0, true>;
+    auto kernel = quant_cols_kernel<true, FMT, SR0, ROT, false, false, QC_FUSED, true, true, SR1>;
+    static PerDeviceOnce setup;
+    static int resident_on[kOnceDevices];
+    int dev = 0;
+    const cudaError_t se = setup.run([&](int d) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Ring::SMEM);
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident_on[d], kernel, QC_THREADS, Ring::SMEM);
+        return e;
+    }, &dev);
+    if (se != cudaSuccess) return se;
+    if (a.rows >= ((int64_t)1 << 31) || a.cols >= ((int64_t)1 << 31) || a.cols % QC_COLS) return cudaErrorInvalidValue;
+    ColTiles ct{};
+    ct.n_tr = (int)((a.rows + QC_ROWS - 1) / QC_ROWS);
+    ct.n_tc = (int)(a.cols / QC_COLS);
+    const int64_t total = (int64_t)ct.n_tr * ct.n_tc;
+    if (total >= ((int64_t)1 << 31) || total == 0) return cudaErrorInvalidValue;
+    ct.total = (int)total;
+    uint32_t l = 0;
+    while (l < 32 && (uint64_t(1) << l) < (uint64_t)ct.n_tc) ++l;
+    ct.tc_m = (uint32_t)((uint64_t)(((unsigned __int128)1 << (32 + l)) / (uint64_t)ct.n_tc) - (uint64_t(1) << 32) + 1);
+    ct.tc_l = l;
+    CUtensorMap tm;
+    if (!make_input_map(&tm, a.x, true, a.rows, a.cols, a.ld, true)) return cudaErrorInvalidValue;
+    const int resident = resident_on[dev];
+    if (resident < 1) return cudaErrorInvalidConfiguration;
+    int64_t grid = (int64_t)num_sms() * resident;
+    if (grid > total) grid = total;
+    QuantArgs ka = a;
+    ColTiles kct = ct;
+    RowOut kro = ro;
+    void* args[] = {&tm, &ka, &kct, &kro};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3((unsigned)grid), dim3(QC_THREADS),
+                                       args, Ring::SMEM, s);
+}
+
+template <int FMT, bool SR0, bool SR1>
+cudaError_t dual_by_rot(const QuantArgs& a, const RowOut& ro, int rot_n, cudaStream_t s) {
+    return rot_n == 16 ? launch_dual_k<FMT, SR0, SR1, 16>(a, ro, s) : launch_dual_k<FMT, SR0, SR1, 0>(a, ro, s);
+}
+
+// entry for fp4_quantize_both_axes (quantize_dual.cu): rot_n 0 or 16, no signs
+inline cudaError_t launch_both_axes_impl(const QuantArgs& a, const RowOut& ro, int fmt, bool sr_cols, bool sr_rows,
+                                         int rot_n, cudaStream_t s) {
+    if (fmt == UFP4) {
+        if (sr_cols) return sr_rows ? dual_by_rot<UFP4, true, true>(a, ro, rot_n, s) : dual_by_rot<UFP4, true, false>(a, ro, rot_n, s);
+        return sr_rows ? dual_by_rot<UFP4, false, true>(a, ro, rot_n, s) : dual_by_rot<UFP4, false, false>(a, ro, rot_n, s);
+    }
+    if (sr_cols) return sr_rows ? dual_by_rot<NVFP4, true, true>(a, ro, rot_n, s) : dual_by_rot<NVFP4, true, false>(a, ro, rot_n, s);
+    return sr_rows ? dual_by_rot<NVFP4, false, true>(a, ro, rot_n, s) : dual_by_rot<NVFP4, false, false>(a, ro, rot_n, s);
 }
 
 // stochastic rounding of a tensor whose column count is not a multiple of 4

@@ -35,7 +35,7 @@ EXPORTS = ("fp4_scales_bytes", "fp4_quantize_workspace_size", "fp4_amax", "fp4_q
            "fp4_gemm", "fp4_last_error", "fp4_status_string", "fp4_set_wait_limit",
            "fp4_quantize_noalloc", "fp4_requantize", "fp4_rotate", "fp4_mxnorm_quantize",
            "fp4_gemm_workspace_size", "fp4_channel_amax", "fp4_outctl_workspace_size", "fp4_outctl_quantize",
-           "fp4_gemm_outctl", "fp4_set_gemm_cta_pairs")
+           "fp4_gemm_outctl", "fp4_set_gemm_cta_pairs", "fp4_quantize_both_axes")
 
 _P, _I, _I64, _U64, _U32, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_uint32, ctypes.c_size_t)
@@ -47,6 +47,8 @@ _lib.fp4_quantize_workspace_size.argtypes = [_I, _I, _I, ctypes.POINTER(_SZ)]
 _lib.fp4_amax.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _P, _P]
 _lib.fp4_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _I, _U64, _U32, _P,
                               _P, _P, _P, _P, _P, _SZ, _P]
+_lib.fp4_quantize_both_axes.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _I, _U32, _P, _P, _P, _I, _U32, _P,
+                                        _P, _P, _P, _SZ, _P]
 _lib.fp4_quantize_noalloc.argtypes = [_P, _I, _I64, _I64, _I64, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P]
 _lib.fp4_requantize.argtypes = [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _I, _I, _U64, _U32, _P, _P, _P, _P, _P,
                                 _P, _SZ, _P]
@@ -66,7 +68,8 @@ _lib.fp4_set_wait_limit.restype = None
 _lib.fp4_set_gemm_cta_pairs.argtypes = [_I]
 _lib.fp4_set_gemm_cta_pairs.restype = None
 for _f in ("fp4_amax", "fp4_rotate", "fp4_mxnorm_quantize", "fp4_gemm_workspace_size", "fp4_channel_amax",
-           "fp4_outctl_workspace_size", "fp4_outctl_quantize", "fp4_gemm_outctl", "fp4_quantize", "fp4_quantize_noalloc", "fp4_requantize", "fp4_gemm", "fp4_last_error",
+           "fp4_outctl_workspace_size", "fp4_outctl_quantize", "fp4_gemm_outctl", "fp4_quantize", "fp4_quantize_noalloc",
+           "fp4_quantize_both_axes", "fp4_requantize", "fp4_gemm", "fp4_last_error",
            "fp4_quantize_workspace_size"):
     getattr(_lib, _f).restype = _I
 
@@ -272,6 +275,34 @@ def quantize(x, fmt, rounding=FP4_RTNE, rotation=FP4_ROT_NONE, axis=1, double_bl
                  tensor_id, tensor_amax, q["codes"], q["scales"], q["outer"], q["tensor_scale"],
                  workspace if ws_bytes else None, ws_bytes, stream)
     return q
+
+
+def fp4_quantize_both_axes(x, in_dtype, rows, cols, ld, fmt, rotation, seed, rounding_rows, tensor_id_rows,
+                           codes_rows, scales_rows, tensor_scale_rows, rounding_cols, tensor_id_cols, codes_cols,
+                           scales_cols, tensor_scale_cols, workspace, workspace_bytes, stream=None) -> None:
+    _check(_lib.fp4_quantize_both_axes(_ptr(x), in_dtype, rows, cols, ld, fmt, rotation, seed, rounding_rows,
+                                       tensor_id_rows, _ptr(codes_rows), _ptr(scales_rows), _ptr(tensor_scale_rows),
+                                       rounding_cols, tensor_id_cols, _ptr(codes_cols), _ptr(scales_cols),
+                                       _ptr(tensor_scale_cols), _ptr(workspace), workspace_bytes, _stream(stream)),
+           "fp4_quantize_both_axes")
+
+
+def quantize_both_axes(x, fmt, rotation=FP4_ROT_NONE, seed=0, rounding_rows=FP4_RTNE, tensor_id_rows=0,
+                       rounding_cols=FP4_RTNE, tensor_id_cols=0, out_rows=None, out_cols=None, workspace=None,
+                       stream=None):
+    """Quantize a 2-D bf16 CUDA tensor along its rows and its columns in one pass;
+    returns (qtensor of the rows, qtensor of the columns)."""
+    import torch
+    rows, cols = x.shape
+    ld = x.stride(0) if rows > 1 else cols
+    qr = out_rows if out_rows is not None else alloc_qtensor(rows, cols, fmt, False, x.device)
+    qc = out_cols if out_cols is not None else alloc_qtensor(cols, rows, fmt, False, x.device)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=x.device)
+    fp4_quantize_both_axes(x, in_dtype_of(x), rows, cols, ld, fmt, rotation, seed, rounding_rows, tensor_id_rows,
+                           qr["codes"], qr["scales"], qr["tensor_scale"], rounding_cols, tensor_id_cols,
+                           qc["codes"], qc["scales"], qc["tensor_scale"], workspace, workspace.numel(), stream)
+    return qr, qc
 
 
 def gemm(qa, qb, out_dtype=FP4_OUT_F32, out=None, workspace=None, stream=None):

@@ -200,6 +200,44 @@ fp4_status_t fp4_quantize(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, 
                           void* stream);
 
 /*
+ * fp4_quantize_both_axes -- fp4_quantize of one tensor along both axes in a
+ * single pass over it.  Every linear layer needs each of its tensors along
+ * both axes: X along its rows for Fprop and along its columns for Wgrad, W
+ * along its rows for Fprop and its columns for Dgrad, dY along its rows for
+ * Dgrad and its columns for Wgrad ("Pre-addestramento di Modelli Linguistici
+ * di Grandi Dimensioni con MXFP4", Metodologia: the three GEMMs of a linear;
+ * "TetraJet-v2" 2.A: the 1x16 groups re-aligned for the transposed operand).
+ * The results are exactly those of two fp4_quantize calls with the internal
+ * tensor amax:
+ *   rows:    axis = 1, rounding_rows, tensor_id_rows -> codes_rows [rows, cols/2],
+ *            scales_rows (fp4_scales_bytes(rows, cols, format)), tensor_scale_rows
+ *   columns: axis = 0, rounding_cols, tensor_id_cols -> codes_cols [cols, rows/2],
+ *            scales_cols (fp4_scales_bytes(cols, rows, format)), tensor_scale_cols
+ * with the same format, rotation and seed.  Each axis has its own rotated
+ * amax and tensor scale.  The tensor is read once from HBM for both amax
+ * passes and once more (mostly from L2) for both quantize passes, in one
+ * cooperative launch whose CTAs meet at a bounded grid barrier.
+ *
+ *   x, in_dtype, rows, cols, ld   as fp4_quantize; in_dtype must be FP4_IN_BF16
+ *   format          FP4_NVFP4 or FP4_UFP4 (no double block)
+ *   rotation        FP4_ROT_NONE or FP4_ROT_H16
+ *   workspace       device, >= 256 bytes (fp4_quantize_workspace_size with the
+ *                   internal amax), 16-byte aligned; contents are scratch
+ * Shape rules: rows % 16 == 0, cols % 64 == 0.  Valid combinations outside the
+ * ones above (f32 input, MXFP4, other rotations) return FP4_ERR_UNSUPPORTED:
+ * use two fp4_quantize calls.  Other errors as fp4_quantize; nothing is
+ * launched on an error.  A grid-barrier or ring wait that runs out sets
+ * FP4_ERR_TIMEOUT for fp4_last_error (the outputs are then not valid).
+ */
+fp4_status_t fp4_quantize_both_axes(const void* x, fp4_in_dtype_t in_dtype, int64_t rows, int64_t cols,
+                                    int64_t ld, fp4_format_t format, fp4_rotation_t rotation, uint64_t seed,
+                                    fp4_rounding_t rounding_rows, uint32_t tensor_id_rows, uint8_t* codes_rows,
+                                    uint8_t* scales_rows, float* tensor_scale_rows,
+                                    fp4_rounding_t rounding_cols, uint32_t tensor_id_cols, uint8_t* codes_cols,
+                                    uint8_t* scales_cols, float* tensor_scale_cols, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
  * fp4_requantize -- re-quantize an already quantized tensor along the other
  * axis.  "TetraJet-v2", section 2.A: the backward pass estimates with X^, the
  * dequantized forward operand, rather than X ("aligning the tensors"), and the

@@ -147,6 +147,31 @@ def test_valid_call_without_gpu_reports_no_device():
     assert g() == fp4.FP4_ERR_NO_DEVICE
 
 
+def both(**kw):
+    a = dict(x=ADDR, dt=fp4.FP4_IN_BF16, rows=256, cols=512, ld=512, fmt=fp4.FP4_NVFP4, rotation=fp4.FP4_ROT_H16,
+             seed=0, rr=fp4.FP4_RTNE, idr=0, cr=ADDR, sr=ADDR, tr=ADDR, rc=fp4.FP4_SR, idc=1, cc=ADDR, sc=ADDR,
+             tc=ADDR, ws=ADDR, wsb=256)
+    a.update(kw)
+    return fp4._lib.fp4_quantize_both_axes(a["x"], a["dt"], a["rows"], a["cols"], a["ld"], a["fmt"], a["rotation"],
+                                           a["seed"], a["rr"], a["idr"], a["cr"], a["sr"], a["tr"], a["rc"], a["idc"],
+                                           a["cc"], a["sc"], a["tc"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dt=5), 1), (dict(fmt=3), 1), (dict(rr=2), 1), (dict(rc=-1), 1), (dict(rotation=9), 1),
+    (dict(x=None), 1), (dict(cr=None), 1), (dict(sc=None), 1), (dict(tr=None), 1), (dict(tc=None), 1),
+    (dict(rows=-1), 1), (dict(ld=500), 1),
+    (dict(dt=fp4.FP4_IN_F32), 8), (dict(fmt=fp4.FP4_MXFP4), 8), (dict(rotation=fp4.FP4_ROT_H32), 8),
+    (dict(rotation=fp4.FP4_ROT_RH16), 8),
+    (dict(cols=480, ld=512), 2), (dict(rows=200), 2),
+    (dict(x=ADDR + 8), 3), (dict(cc=ADDR + 4), 3), (dict(tr=ADDR + 2), 3),
+    (dict(ws=None), 4), (dict(wsb=16), 4),
+    (dict(), fp4.FP4_ERR_NO_DEVICE),
+])
+def test_quantize_both_axes_host_validation(kw, status):
+    assert both(**kw) == status
+
+
 def rot(**kw):
     a = dict(x=ADDR, dt=fp4.FP4_IN_BF16, rows=64, cols=256, ld=256, rotation=fp4.FP4_ROT_H16, axis=1, seed=0,
              y=ADDR, ldy=256)
