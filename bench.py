@@ -680,6 +680,21 @@ def measure_configs(fp4, device, peaks, layer=None, reps=10, only=CONFIG_NAMES):
                              "gemm": ug, "gemm_total_ms": g_ms, "gemm_tflops": g_flop / (g_ms * 1e-3) / 1e12,
                              "gemm_frac_fp4_over_4": g_flop / (g_ms * 1e-3) / 1e12 / (fp4_peak / 4)}
         del ws
+        # the same 24 UFP4 operands from 12 both-axes calls
+        both_ms = 0.0
+        wsb = torch.empty(256, dtype=torch.uint8, device=device)
+        for lin in layer.linears:
+            for b in lin["both"]:
+                x = lin["t"][b["x"]]
+                cr, cc = lin["calls"][b["rows"]], lin["calls"][b["cols"]]
+                R, C = x.shape
+                qr, qc = fp4.alloc_qtensor(R, C, UF, False, device), fp4.alloc_qtensor(C, R, UF, False, device)
+                both_ms += _median_ms(lambda: fp4.quantize_both_axes(
+                    x, UF, fp4.FP4_ROT_H16, seed=0, rounding_rows=cr["rounding"], tensor_id_rows=cr["tensor_id"],
+                    rounding_cols=cc["rounding"], tensor_id_cols=cc["tensor_id"], out_rows=qr, out_cols=qc,
+                    workspace=wsb), flush, reps)
+                del qr, qc
+        out["ufp4_layer"]["quantize_both_axes_total_ms"] = both_ms
 
     if "mxnorm" in only and layer is not None:
         # MXNorm fused with the cast ("MXNorm: Reusing MXFP block scales...":

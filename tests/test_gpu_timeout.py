@@ -98,3 +98,30 @@ def test_one_launch_quantizer_wait_timeout_is_reported_and_recoverable(fp4, fmt,
         assert torch.equal(before[key].view(torch.uint8), after[key].view(torch.uint8)), key
     n = fp4.fp4_scales_bytes(8192, 4096, kw["fmt"])
     assert torch.equal(before["scales"][:n], after["scales"][:n])
+
+
+# The both-axes quantizer (column kernel with the row part) runs the same
+# bounded ring and grid-barrier waits; at one poll they run out, the call is
+# reported, and the next call at the default limit gives the earlier bytes.
+def test_both_axes_quantizer_wait_timeout_is_reported_and_recoverable(fp4):
+    g = torch.Generator().manual_seed(12)
+    x = torch.randn((8192, 4096), generator=g).to(torch.bfloat16).cuda()
+    kw = dict(fmt=fp4.FP4_NVFP4, rotation=1, seed=3, rounding_rows=0, tensor_id_rows=1, rounding_cols=1,
+              tensor_id_cols=2)
+    before = fp4.quantize_both_axes(x, **kw)
+    torch.cuda.synchronize()
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+
+    fp4.fp4_set_wait_limit(1)
+    try:
+        fp4.quantize_both_axes(x, **kw)
+        status = fp4.fp4_last_error()
+    finally:
+        fp4.fp4_set_wait_limit(0)
+    assert status == fp4.FP4_ERR_TIMEOUT, fp4.fp4_status_string(status)
+
+    after = fp4.quantize_both_axes(x, **kw)
+    assert fp4.fp4_last_error() == fp4.FP4_OK
+    for b, a in zip(before, after):
+        for key in ("codes", "scales", "tensor_scale"):
+            assert torch.equal(b[key].view(torch.uint8), a[key].view(torch.uint8)), key
