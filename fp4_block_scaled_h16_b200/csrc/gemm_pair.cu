@@ -84,17 +84,39 @@ struct PairParams {
     const float* b_ts;
     int K;
     int tiles_m, tiles_n;    // pair tiles
+    // work units: tiles [0, split_base) whole; the tiles after it (a last wave
+    // that would keep at most half the pairs busy) as two 256 x 128 halves
+    int units, split_base;
     uint32_t wait_limit;
     unsigned int* err;
 };
+
+// output block of work unit u: rows m0 .. m0+255, columns n0 .. (256 of them,
+// or 128 for a half unit)
+__device__ __forceinline__ bool pair_unit(const PairParams& p, int u, int& m0, int& n0) {
+    int tm, tn;
+    if (u < p.split_base) {
+        tile_coords(u, p.tiles_m, p.tiles_n, tm, tn);
+        m0 = tm * PM;
+        n0 = tn * PN;
+        return false;
+    }
+    const int t = p.split_base + ((u - p.split_base) >> 1);
+    tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+    m0 = tm * PM;
+    n0 = tn * PN + ((u - p.split_base) & 1) * (PN / 2);
+    return true;
+}
 
 __device__ __forceinline__ void raise_timeout(const PairParams& p, volatile int* abort_flag) {
     *abort_flag = 1;
     atomicExch(p.err, ERR_TIMEOUT);
 }
 
-// one stage's scale copies and MMAs, issued by the leader for both CTAs
-template <int FMT>
+// one stage's scale copies and MMAs, issued by the leader for both CTAs;
+// NMMA = 256, or 128 for a half unit (each CTA's first 64 rows of B; the
+// scales of its 128 columns are the first of the two row blocks copied)
+template <int FMT, int NMMA>
 __device__ __forceinline__ void mma_stage_pair(uint32_t tmem, uint32_t st, int kt) {
     using G = PCfg<FMT>;
     const uint32_t st_sfa = st + G::A_BYTES + G::B_BYTES;
@@ -114,10 +136,10 @@ __device__ __forceinline__ void mma_stage_pair(uint32_t tmem, uint32_t st, int k
         const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
         if (FMT == MXFP4) {
             const int j = kk / 2;
-            const uint32_t id = sm100::idesc_block_scaled(PN, true, (kk & 1) * 2, (kk & 1) * 2, PM);
+            const uint32_t id = sm100::idesc_block_scaled(NMMA, true, (kk & 1) * 2, (kk & 1) * 2, PM);
             sm100::mma_mxf4_pair(tmem, da, db, id, tmem + G::SFA_COL + 4 * j, tmem + G::SFB_COL + 8 * j, acc);
         } else {
-            const uint32_t id = sm100::idesc_block_scaled(PN, false, 0, 0, PM);
+            const uint32_t id = sm100::idesc_block_scaled(NMMA, false, 0, 0, PM);
             sm100::mma_nvf4_pair(tmem, da, db, id, tmem + G::SFA_COL + 4 * kk, tmem + G::SFB_COL + 8 * kk, acc);
         }
     }
@@ -148,7 +170,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = sm100::cluster_rank();
     const int pair = (int)(blockIdx.x >> 1), pairs = (int)(gridDim.x >> 1);
-    const int units = p.tiles_m * p.tiles_n;
+    const int units = p.units;
     const int kt_count = (p.K + BK - 1) / BK;   // a ragged last stage reads zeros past K
 
     if (threadIdx.x == 0) {
@@ -186,10 +208,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t fills = 0;           // fill i went to stage i % STAGES, phase i / STAGES
             bool ok = true;
             for (int u = pair; u < units && ok; u += pairs) {
-                int tm, tn;
-                tile_coords(u, p.tiles_m, p.tiles_n, tm, tn);
-                const int ma = tm * PM + 128 * (int)rank;     // this CTA's rows of A
-                const int nb = tn * PN;                       // first column of the tile
+                int m0, nb;                                   // first row and column of the unit
+                const bool half_unit = pair_unit(p, u, m0, nb);
+                const int ma = m0 + 128 * (int)rank;          // this CTA's rows of A
+                // this CTA's rows of B: 128 of a whole tile; for a half unit the
+                // MMA reads the first 64 of the box (the rest, past the unit or
+                // zero-filled past N, keeps every fill the same size)
+                const int nbc = nb + (half_unit ? 64 : 128) * (int)rank;
                 for (int kt = 0; kt < kt_count; ++kt) {
                     if (!sm100::mbar_wait(&empty[stage], phase ^ 1u, p.wait_limit, abort_flag)) {
                         raise_timeout(p, abort_flag);
@@ -200,7 +225,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const uint32_t bar = sm100::cluster_addr(&full[stage], 0);
                     if (rank == 0) sm100::mbar_arrive_expect_tx(&full[stage], 2 * G::STAGE_BYTES);
                     sm100::tma_load_2d_pair(st, &tmA, kt * (BK / 2), ma, bar);
-                    sm100::tma_load_2d_pair(st + G::A_BYTES, &tmB, kt * (BK / 2), nb + 128 * (int)rank, bar);
+                    sm100::tma_load_2d_pair(st + G::A_BYTES, &tmB, kt * (BK / 2), nbc, bar);
                     sm100::tma_load_3d_pair(st + G::A_BYTES + G::B_BYTES, &tmSA, 0, kt * 2 * G::ATOMS, ma / 128, bar);
                     sm100::tma_load_3d_pair(st + G::A_BYTES + G::B_BYTES + G::SFA_BYTES, &tmSB, 0,
                                             kt * 2 * G::ATOMS, nb / 128, bar);
@@ -249,6 +274,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, issued = false;
             for (int u = pair; u < units && ok; u += pairs) {
+                const bool half_unit = u >= p.split_base;
                 if (!sm100::mbar_wait_cluster(acc_empty, acc_phase ^ 1u, p.wait_limit, abort_flag)) {
                     raise_timeout(p, abort_flag);
                     break;
@@ -261,7 +287,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         break;
                     }
                     sm100::tc_fence_after();
-                    mma_stage_pair<FMT>(tmem, sm100::smem_u32(smem + stage * G::STAGE_BYTES), kt);
+                    const uint32_t st = sm100::smem_u32(smem + stage * G::STAGE_BYTES);
+                    if (half_unit) mma_stage_pair<FMT, PN / 2>(tmem, st, kt);
+                    else mma_stage_pair<FMT, PN>(tmem, st, kt);
                     issued = true;
                     sm100::tc_commit_pair_both(&empty[stage]);   // both CTAs' stage free once these MMAs are done
                     if (++stage == G::STAGES) { stage = 0; phase ^= 1u; }
@@ -289,8 +317,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const uint32_t leader_acc_empty = sm100::cluster_addr(acc_empty, 0);
         uint32_t acc_phase = 0;
         for (int u = pair; u < units; u += pairs) {
-            int tm, tn;
-            tile_coords(u, p.tiles_m, p.tiles_n, tm, tn);
+            int m0, nu;
+            const bool half_unit = pair_unit(p, u, m0, nu);
+            // a half unit has 128 columns: the second column half's warps only hand over
+            const bool idle = half_unit && half == 1;
             int got = 0;
             if (lane == 0) {
                 got = sm100::mbar_wait(acc_full, acc_phase, p.wait_limit, abort_flag) ? 1 : 0;
@@ -299,19 +329,22 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
             sm100::tc_fence_after();
             uint32_t r[COLS];
+            if (!idle) {
 #pragma unroll
-            for (int c = 0; c < COLS / 32; ++c) {
-                uint32_t (&rr)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[32 * c]);
-                sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + half * COLS + 32 * c, rr);
+                for (int c = 0; c < COLS / 32; ++c) {
+                    uint32_t (&rr)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[32 * c]);
+                    sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + half * COLS + 32 * c, rr);
+                }
+                sm100::tmem_ld_wait();
             }
-            sm100::tmem_ld_wait();
             sm100::tc_fence_before();
             __syncwarp();
             if (lane == 0) sm100::mbar_arrive_cluster(leader_acc_empty);   // the MMA may overwrite it now
             acc_phase ^= 1u;
+            if (idle) continue;
             // rows row0 .. row0 + 31 (lane = row), columns n0 .. n0 + COLS - 1
-            const int row0 = tm * PM + 128 * (int)rank + 32 * q;
-            const int n0 = tn * PN + half * COLS;
+            const int row0 = m0 + 128 * (int)rank + 32 * q;
+            const int n0 = nu + half * COLS;
 #pragma unroll
             for (int b = 0; b < COLS / BOX_COLS; ++b) {
                 if (lane == 0) sm100::bulk_wait_read0();        // the previous box has left the buffer
@@ -409,6 +442,12 @@ cudaError_t run_pair(const GemmArgs& g, cudaStream_t s) {
     p.err = device_error_word();
     const int tiles = p.tiles_m * p.tiles_n;
     const int pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+    // a last wave that would leave more than half the pairs idle runs as half
+    // tiles, so the tail takes about half as long
+    const int full_waves = tiles / pairs, tail = tiles - full_waves * pairs;
+    const bool split = full_waves > 0 && tail > 0 && 2 * tail <= pairs;
+    p.split_base = split ? full_waves * pairs : tiles;
+    p.units = split ? p.split_base + 2 * tail : tiles;
     gemm_pair_kernel<FMT, OUT_BF16><<<2 * pairs, NUM_THREADS, G::SMEM, s>>>(ta, tb, tsa, tsb, tc, p);
     return cudaGetLastError();
 }

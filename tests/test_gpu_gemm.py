@@ -62,25 +62,29 @@ def test_gemm_on_oracle_operands(fp4, fmt, out_bf16, shape, cta_pairs):
 
 
 @pytest.mark.parametrize("fmt", [MX, NV])
-@pytest.mark.parametrize("shape", [(5120, 1024, 256), (2560, 2048, 512), (5120, 1024, 384)])
-def test_gemm_with_more_tiles_than_sms_on_oracle_operands(fp4, fmt, shape, cta_pairs):
+@pytest.mark.parametrize("out_bf16", [True, False])
+@pytest.mark.parametrize("shape", [(5120, 1024, 256), (2560, 2048, 512), (5120, 1024, 384), (4096, 5120, 256)])
+def test_gemm_with_more_tiles_than_sms_on_oracle_operands(fp4, fmt, shape, out_bf16, cta_pairs):
     # single CTAs: more 128x256 tiles than SMs (160 tiles on 148 SMs: a
     # second, nearly empty wave of persistent tiles, run as 128-column halves;
     # K = 384 ends on a half stage).  CTA pairs: 80 256x256 tiles on 74 pairs,
-    # a second wave of 6.  Every element against the oracle.
+    # a second wave of 6, run as 256x128 halves; 4096 x 5120: 320 pair tiles,
+    # a last wave of 24 as 48 halves (640 single tiles, a last wave of 48 as
+    # 96 halves).  Every element against the oracle.
     M, N, K = shape
     a, b = rand(M, K, M + fmt), rand(N, K, N + 7 + fmt, 0.1)
     qa = oracle_quantize(a, fmt=fmt)
     qb = oracle_quantize(b, fmt=fmt)
     C64, bound = oracle.gemm(qa, qb)
-    C = fp4.gemm(upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb), fp4.FP4_OUT_BF16)
+    C = fp4.gemm(upload_oracle_qtensor(fp4, qa), upload_oracle_qtensor(fp4, qb),
+                 fp4.FP4_OUT_BF16 if out_bf16 else fp4.FP4_OUT_F32)
     torch.cuda.synchronize()
     assert fp4.fp4_last_error() == fp4.FP4_OK
-    assert_within_gemm_bound(C.float().cpu().numpy(), C64, bound, True, what=str((fmt, shape)))
+    assert_within_gemm_bound(C.float().cpu().numpy(), C64, bound, out_bf16, what=str((fmt, shape, out_bf16)))
 
 
 @pytest.mark.parametrize("fmt", [MX, NV])
-@pytest.mark.parametrize("shape", [(512, 512, 1024), (2048, 1536, 640)])
+@pytest.mark.parametrize("shape", [(512, 512, 1024), (2048, 1536, 640), (5120, 1024, 384)])
 def test_pair_and_single_cta_tiles_give_the_same_bits(fp4, fmt, shape):
     """The pair MMA (M = 256 over two SMs) and the single-CTA MMA (M = 128)
     take the same 64-element K slices in the same order for every output, so
