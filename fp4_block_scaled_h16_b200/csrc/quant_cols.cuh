@@ -54,13 +54,16 @@ __device__ __forceinline__ uint32_t qc_grid_limit(uint32_t w) { return w >= (1u 
 
 // Four CTAs per SM (128 registers).  (Measured on B200: a fifth CTA for the
 // stochastic-rounding variants, at 96 registers with two stages, was no
-// faster: they are bound by their instruction count, not by occupancy.)
+// faster: they are bound by their instruction count, not by occupancy.)  The
+// both-axes variants with stochastic rounding on the columns run three CTAs
+// per SM: at 128 registers they spilled, and with up to 168 they are 7%
+// faster on the layer's tensors; two CTAs, or a fourth stage, were slower.
 template <bool BF16, bool SR, bool SWZ = false>
 struct ColRing {
     static constexpr int ES = BF16 ? 2 : 4;
     static constexpr int BYTES = QC_ROWS * QC_COLS * ES;        // one tile: 16 KB (bf16) / 32 KB (f32)
     static constexpr int STAGES = BF16 ? 3 : 2;
-    static constexpr int CTAS = 4;                              // the launch bound
+    static constexpr int CTAS = (SWZ && SR) ? 3 : 4;            // the launch bound
     static constexpr int ALIGN = SWZ ? 1024 : 128;              // the 128-byte swizzle wants 1024-byte stages
     static constexpr int SMEM = STAGES * BYTES + ALIGN /*alignment*/ + STAGES * 16 /*barriers*/;
 };
@@ -351,27 +354,31 @@ quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, co
                     }
                 }
             }
-            const float cn = (ROT == 16) ? 0.25f : __uint_as_float(0x3E3504F3u);   // binary32(1/sqrt(32))
-            const float2 cc = make_float2(cn, cn);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                v[j][0] = mul2(v[j][0], cc);
-                v[j][1] = mul2(v[j][1], cc);
-            }
         }
+        const float cn = (ROT == 16) ? 0.25f : __uint_as_float(0x3E3504F3u);   // binary32(1/sqrt(32))
 
-        // ---- column maxima of my 16 rows
+        // ---- column maxima of my 16 rows; with a rotation they are taken before
+        // the factor c_n and scaled after: max |RN(c y)| = RN(c max |y|), since
+        // c > 0 and rounding are monotone, so the amax pass skips the 64 products
         float m[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             float mm = 0.0f;
 #pragma unroll
             for (int j = 0; j + 1 < 16; j += 2) mm = amax3(mm, col_of(v[j][c >> 1], c), col_of(v[j + 1][c >> 1], c));
-            m[c] = mm;
+            m[c] = ROT ? __fmul_rn(mm, cn) : mm;
         }
         if (AMAX_ONLY || (FUSED && it < n)) {
             tmax = fmaxf(tmax, fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])));
             continue;
+        }
+        if (ROT) {
+            const float2 cc = make_float2(cn, cn);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                v[j][0] = mul2(v[j][0], cc);
+                v[j][1] = mul2(v[j][1], cc);
+            }
         }
 
         const int tr = (int)fast_div((uint32_t)t, ct.tc_m, ct.tc_l), tc = t - tr * ct.n_tc;
