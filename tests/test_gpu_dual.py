@@ -141,3 +141,17 @@ def test_both_axes_layer_sizes(fp4, name):
         assert_quant_equal(hc, oracle_quantize(d[tn], NV, rounding=kw["rounding_cols"], rotation=1, axis=0, seed=0,
                                                tensor_id=kw["tensor_id_cols"], lines=lc), lines=lc,
                            what="%s.%s columns" % (name, tn))
+
+
+@pytest.mark.parametrize("shape", [(16, 64), (144, 128), (48, 192), (272, 64)])
+@pytest.mark.parametrize("rr,rc", [(0, 1), (1, 0)])
+def test_both_axes_small_and_ragged(fp4, shape, rr, rc):
+    # fewer rows than one 128-row tile, a ragged second tile, one column tile
+    R, C = shape
+    x = make_input(R, C, 7 * R + C + rr)
+    kw = dict(fmt=NV, rotation=1, seed=11, rounding_rows=rr, tensor_id_rows=3, rounding_cols=rc, tensor_id_cols=4)
+    qr, qc = both(fp4, x.cuda(), **kw)
+    assert_quant_equal(host(qr), oracle_quantize(x, NV, rounding=rr, rotation=1, axis=1, seed=11, tensor_id=3),
+                       what="rows %s" % (shape,))
+    assert_quant_equal(host(qc), oracle_quantize(x, NV, rounding=rc, rotation=1, axis=0, seed=11, tensor_id=4),
+                       what="columns %s" % (shape,))
