@@ -46,10 +46,10 @@ GEMMS = workloads.LAYER_GEMMS
 # averaged over the 12 GEMM launches of one layer step, from one ncu capture of
 # the current kernel (profiles/gemm_layer_llama8b_t8192.md); the algorithmic
 # bytes (operands read once, C written once) average 241.7 MB
-GEMM_TRAFFIC_BYTES_PER_LAUNCH = 276_684_800
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = 276_598_528
 # the same for the step's 12 both-axes quantize launches (profiles/quant_both_axes_layer_llama8b_t8192.md);
 # their algorithmic bytes (input read twice, both outputs written) average 336.8 MB
-QUANT_BOTH_TRAFFIC_BYTES_PER_LAUNCH = 251_938_901
+QUANT_BOTH_TRAFFIC_BYTES_PER_LAUNCH = 246_176_917
 
 
 class L2Flush:
@@ -565,8 +565,8 @@ def finish_line(args, rank, world, device, layer, fam, table, total_ms, e2e_ms, 
                 "traffic_is": ("ncu DRAM read + write bytes per launch, averaged over the step's 12 both-axes "
                                "launches (algorithmic average 336.8 MB: the second read of a tensor that fits in "
                                "L2 comes from L2)" if dom == "quant_both" else None),
-                "bound_by": ("instruction issue: 60 thread instructions per element at 50% issue for a call with "
-                             "SR columns, 7.6% of DRAM throughput (ncu)" if dom == "quant_both" else None),
+                "bound_by": ("instruction issue: 59 thread instructions per element at 51% issue for a call with "
+                             "SR columns, 7.8% of DRAM throughput (ncu)" if dom == "quant_both" else None),
                 "achieved_is": "algorithmic bytes (input read twice: amax pass + quantize; codes and "
                                "scales written) / summed mean event time",
                 "peak_is": "%s HBM copy bandwidth" % peaks["src"]}
