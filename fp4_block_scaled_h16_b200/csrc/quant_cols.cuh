@@ -30,9 +30,11 @@
 // at chunk c ^ (r % 8)), so that thread t reading tile row t (two 32-element
 // row units, the row quantizer's arithmetic) and the column lanes both read
 // shared memory without bank conflicts.  The row part of each tile runs
-// before the column part copies the tile out and releases its slot.  Every wait is bounded by the
-// wait limit of fp4_set_wait_limit (ring: 16 x, grid barrier: 4 x); whatever
-// way a CTA leaves, thread 0 first waits for every tile load it issued.
+// before the column part copies the tile out and releases its slot.
+//
+// Every wait is bounded by the wait limit of fp4_set_wait_limit (ring: 16 x,
+// grid barrier: 4 x); whatever way a CTA leaves, thread 0 first waits for
+// every tile load it issued.
 #pragma once
 
 #include <cuda.h>
@@ -67,7 +69,6 @@ struct ColRing {
     static constexpr int ALIGN = SWZ ? 1024 : 128;              // the 128-byte swizzle wants 1024-byte stages
     static constexpr int SMEM = STAGES * BYTES + ALIGN /*alignment*/ + STAGES * 16 /*barriers*/;
 };
-
 
 struct ColTiles {
     int n_tr, n_tc, total;      // row tiles, column tiles, n_tr * n_tc (< 2^31)
