@@ -60,6 +60,9 @@ __device__ __forceinline__ uint32_t qc_grid_limit(uint32_t w) { return w >= (1u 
 // both-axes variants with stochastic rounding on the columns run three CTAs
 // per SM: at 128 registers they spilled, and with up to 168 they are 7%
 // faster on the layer's tensors; two CTAs, or a fourth stage, were slower.
+// The double-block variants (about 150 bytes of spills at 128 registers) run
+// three CTAs per SM as well: 8% faster on a 4096 x 14336 weight.  (MXFP4 with
+// stochastic rounding measured slower at three.)
 template <bool BF16, bool SR, bool SWZ = false>
 struct ColRing {
     static constexpr int ES = BF16 ? 2 : 4;
@@ -98,7 +101,7 @@ __device__ __forceinline__ float col_of(const float2& p, int c) { return (c & 1)
 // DUAL / SR1: also quantize along the rows (rounding SR1), see the file comment
 template <bool BF16, int FMT, bool SR, int ROT, bool SIGNS, bool DB, int MODE, bool ALIGN4 = true, bool DUAL = false,
           bool SR1 = false>
-__global__ void __launch_bounds__(QC_THREADS, (ColRing<BF16, SR, DUAL>::CTAS))
+__global__ void __launch_bounds__(QC_THREADS, (DB ? 3 : ColRing<BF16, SR, DUAL>::CTAS))
 quant_cols_kernel(const __grid_constant__ CUtensorMap tmx, const QuantArgs a, const ColTiles ct, const RowOut ro) {
     constexpr bool AMAX_ONLY = MODE == QC_AMAX, FUSED = MODE == QC_FUSED;
     static_assert(!FUSED || (FMT != MXFP4 && !DB), "only a tensor-scaled format has an amax pass");
